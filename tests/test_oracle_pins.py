@@ -1,0 +1,423 @@
+"""Pins for the CPU oracle: each check fixes the oracle to something other than
+itself -- hand-computed fixtures, closed forms, invariants, exact rational brute
+force, and library conversions -- so that a dropped term, a wrong sign or
+index, or a transposed operand anywhere in the oracle fails one of them.
+CPU only."""
+from __future__ import annotations
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import q8gen
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --------------------------------------------------------------------------
+# binary16 conversions, pinned to numpy's float16 (a library routine)
+# --------------------------------------------------------------------------
+
+def test_half_decode_matches_numpy_all_patterns():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.half_to_double(int(b)) for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    # signed zero survives
+    assert math.copysign(1.0, oracle.half_to_double(0x8000)) == -1.0
+
+
+def _encode_cases():
+    rng = np.random.default_rng(7)
+    halves = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)
+    mids = (halves[:-1] + halves[1:]) / 2  # exact ties between neighbours
+    vals = np.concatenate([
+        halves, mids, np.nextafter(mids, 0), np.nextafter(mids, 1),
+        rng.standard_normal(20000) * 0.02,
+        np.exp(rng.uniform(-20, 11.2, 20000)),
+        [65504, 65519.99, 65520, 65536, 1e9, 2.0 ** -24, 2.0 ** -25, 2.0 ** -26, 3 * 2.0 ** -26],
+    ])
+    vals = vals.astype(np.float32)
+    return np.concatenate([vals, -vals])
+
+
+def test_half_encode_matches_numpy():
+    vals = _encode_cases()
+    with np.errstate(over="ignore"):
+        ref = vals.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.float_to_half_rn(float(v)) for v in vals], np.uint16)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, f"{bad.size} mismatches, e.g. {vals[bad[:5]]}"
+
+
+# --------------------------------------------------------------------------
+# GGUF block layout (hand-written bytes)
+# --------------------------------------------------------------------------
+
+def _read_layout():
+    entries, cur = [], {}
+    for line in open(os.path.join(GOLDEN, "q8_0_block_layout.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        key, val = line.split(":", 1)
+        cur[key.strip()] = val.split()
+        if key.strip() == "q":
+            entries.append(cur)
+            cur = {}
+    return entries
+
+
+def test_block_layout_decodes_as_written():
+    for e in _read_layout():
+        raw = np.array([int(b, 16) for b in e["bytes"]], np.uint8)
+        assert raw.size == 34
+        d = float(e["d"][0])
+        q = np.array([int(v) for v in e["q"]], np.int64)
+        # Decode through the oracle's GEMV with one-hot activations: y_k = d * q_k.
+        for k in range(32):
+            x = np.zeros((1, 32), np.float32)
+            x[0, k] = 1.0
+            y, _ = oracle.gemv(raw, x, 1, 32)
+            assert y[0, 0] == d * q[k]
+        # ...and the generator's assembler writes the same bytes back.
+        dbits = np.array([[int(raw[0]) | (int(raw[1]) << 8)]], np.uint16)
+        again = q8gen.assemble_gguf(q.astype(np.int8).reshape(1, 32), dbits)
+        assert np.array_equal(again, raw)
+
+
+# --------------------------------------------------------------------------
+# P5: hand-computed blocks
+# --------------------------------------------------------------------------
+
+def _hand_blocks():
+    out = []
+    for line in open(os.path.join(GOLDEN, "hand_blocks.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        d, q, x, y = [p.split() for p in line.split("|")]
+        out.append((float(d[0]), [int(v) for v in q], [float(v) for v in x], float(y[0])))
+    return out
+
+
+@pytest.mark.parametrize("case", range(4))
+def test_hand_blocks(case):
+    d, q, x, y = _hand_blocks()[case]
+    dbits = np.array([[np.float16(d).view(np.uint16)]], np.uint16)
+    g = q8gen.assemble_gguf(np.array([q], np.int8), dbits)
+    got, gabs = oracle.gemv(g, np.array([x], np.float32), 1, 32)
+    assert got[0, 0] == y
+    assert gabs[0, 0] == sum(abs(d * qi * xi) for qi, xi in zip(q, x))
+
+
+# --------------------------------------------------------------------------
+# P1: brute force with exact rationals on tiny shapes
+# --------------------------------------------------------------------------
+
+def _exact_gemv(gguf, x, M, K):
+    q, dbits = q8gen.split_gguf(gguf, M, K)
+    d = dbits.view(np.float16).astype(np.float64)
+    N = x.shape[0]
+    y = [[Fraction(0)] * M for _ in range(N)]
+    for n in range(N):
+        for m in range(M):
+            s = Fraction(0)
+            for k in range(K):
+                s += Fraction(float(d[m, k // 32])) * int(q[m, k]) * Fraction(float(x[n, k]))
+            y[n][m] = s
+    return y
+
+
+@pytest.mark.parametrize("M,K,N,seed", [(1, 32, 1, 1), (3, 64, 2, 2), (4, 32, 3, 3), (2, 96, 1, 4)])
+def test_brute_force_gemv(M, K, N, seed):
+    g, x = q8gen.q8_matrix(seed, M, K, N)
+    y, ya = oracle.gemv(g, x, M, K)
+    exact = _exact_gemv(g, x, M, K)
+    for n in range(N):
+        for m in range(M):
+            e = exact[n][m]
+            assert abs(Fraction(y[n, m]) - e) <= Fraction(ya[n, m]) * Fraction(2, 2 ** 52)
+
+
+def test_brute_force_gate_up_g_u():
+    I, K = 3, 64
+    g8, x = q8gen.q8_matrix(11, 2 * I, K, 2)
+    out = oracle.gate_up_swiglu(g8, x, I, K)
+    exact = _exact_gemv(g8, x, 2 * I, K)
+    for n in range(2):
+        for i in range(I):
+            assert abs(Fraction(out["g"][n, i]) - exact[n][i]) <= Fraction(out["g_abs"][n, i]) / 2 ** 51
+            assert abs(Fraction(out["u"][n, i]) - exact[n][I + i]) <= Fraction(out["u_abs"][n, i]) / 2 ** 51
+
+
+def test_brute_force_q8q8():
+    M, K, N = 3, 64, 2
+    g, x = q8gen.q8_matrix(21, M, K, N)
+    xq, xd, _ = oracle.quantize_act(x)
+    dots, y, ya = oracle.q8q8(g, xq, xd, M, K)
+    q, dbits = q8gen.split_gguf(g, M, K)
+    dw = dbits.view(np.float16).astype(np.float64)
+    dx = xd.view(np.float16).astype(np.float64)
+    for n in range(N):
+        for m in range(M):
+            tot = Fraction(0)
+            for b in range(K // 32):
+                dot = sum(int(q[m, b * 32 + i]) * int(xq[n, b * 32 + i]) for i in range(32))
+                assert dots[n, m, b] == dot
+                tot += Fraction(float(dw[m, b])) * Fraction(float(dx[n, b])) * dot
+            assert abs(Fraction(y[n, m]) - tot) <= Fraction(ya[n, m]) / 2 ** 51
+
+
+# --------------------------------------------------------------------------
+# P2: closed form -- unit scales and one-hot x return a column of q exactly
+# --------------------------------------------------------------------------
+
+def test_one_hot_returns_column():
+    M, K = 5, 96
+    rng = np.random.default_rng(5)
+    q = rng.integers(-127, 128, (M, K), dtype=np.int8)
+    dbits = np.full((M, K // 32), 0x3C00, np.uint16)  # d = 1.0
+    g = q8gen.assemble_gguf(q, dbits)
+    for k in (0, 31, 32, 95):
+        x = np.zeros((1, K), np.float32)
+        x[0, k] = 1.0
+        y, _ = oracle.gemv(g, x, M, K)
+        assert np.array_equal(y[0], q[:, k].astype(np.float64))
+
+
+def test_row_and_column_orientation():
+    """x column n and output row m are not transposed: distinct rows and
+    distinct activation vectors give distinct, correctly placed results."""
+    M, K = 2, 32
+    q = np.zeros((M, K), np.int8)
+    q[0, 0] = 1      # row 0 picks x[:, 0]
+    q[1, 1] = 1      # row 1 picks x[:, 1]
+    g = q8gen.assemble_gguf(q, np.full((M, 1), 0x3C00, np.uint16))
+    x = np.zeros((3, K), np.float32)
+    x[:, 0] = [1, 2, 3]
+    x[:, 1] = [10, 20, 30]
+    y, _ = oracle.gemv(g, x, M, K)
+    assert np.array_equal(y, [[1, 10], [2, 20], [3, 30]])
+
+
+# --------------------------------------------------------------------------
+# P3: linearity in d and x
+# --------------------------------------------------------------------------
+
+def test_linearity():
+    M, K = 7, 128
+    g, x = q8gen.q8_matrix(31, M, K, 2)
+    y, ya = oracle.gemv(g, x, M, K)
+    # doubling every d (exact in binary16 away from the top of the range)
+    q, dbits = q8gen.split_gguf(g, M, K)
+    d2 = (dbits.view(np.float16).astype(np.float32) * 2).astype(np.float16).view(np.uint16)
+    y2, _ = oracle.gemv(q8gen.assemble_gguf(q, d2), x, M, K)
+    assert np.array_equal(y2, 2 * y)
+    # doubling x
+    y3, _ = oracle.gemv(g, 2 * x, M, K)
+    assert np.array_equal(y3, 2 * y)
+    # additivity
+    xa = q8gen.activations(1, 2, K)
+    xb = q8gen.activations(2, 2, K)
+    ya_, aa = oracle.gemv(g, xa, M, K)
+    yb_, ab = oracle.gemv(g, xb, M, K)
+    xs = (xa.astype(np.float64) + xb).astype(np.float32)
+    ys, _ = oracle.gemv(g, xs, M, K)
+    # x_a + x_b is rounded to fp32 once per element: bound that, plus fp64 sums
+    rounding = oracle.gemv(q8gen.assemble_gguf(np.abs(q.astype(np.int16)).astype(np.int8), dbits),
+                           np.abs(xs), M, K)[0] * 2.0 ** -24
+    assert np.all(np.abs(ys - (ya_ + yb_)) <= rounding + 1e-12 * (aa + ab))
+    # negating q flips the sign exactly
+    yn, _ = oracle.gemv(q8gen.assemble_gguf(-q, dbits), x, M, K)
+    assert np.array_equal(yn, -y)
+
+
+# --------------------------------------------------------------------------
+# P4: Q8_0 round trip |w - d*q| <= d/2
+# --------------------------------------------------------------------------
+
+def test_round_trip_bound():
+    rng = np.random.default_rng(9)
+    M, K = 16, 256
+    w = (rng.standard_normal((M, K)) * np.exp(rng.uniform(-8, 4, (M, 1)))).astype(np.float32)
+    w[3, 32:64] = 0.0  # an all-zero block
+    gguf, d32 = oracle.quantize_weights(w)
+    q, dbits = q8gen.split_gguf(gguf, M, K)
+    d = np.repeat(d32.astype(np.float64), 32, axis=1)
+    err = np.abs(w.astype(np.float64) - d * q)
+    # d32 and w/d32 are fp32-rounded: allow their rounding on top of d/2
+    assert np.all(err <= d / 2 * (1 + 2.0 ** -20))
+    assert np.all(q[3, 32:64] == 0) and dbits[3, 1] == 0
+    # the largest |w| of a block maps to +-127
+    blk = np.abs(w.reshape(M, K // 32, 32)).argmax(axis=2)
+    qb = np.abs(q.reshape(M, K // 32, 32))
+    pick = np.take_along_axis(qb, blk[..., None], 2)[..., 0]
+    nz = d32 > 0
+    assert np.all(pick[nz] == 127)
+    # stored scale is binary16(d32)
+    assert np.array_equal(dbits, d32.astype(np.float16).view(np.uint16))
+
+
+# --------------------------------------------------------------------------
+# P6: activation quantisation -- hand blocks and invariants
+# --------------------------------------------------------------------------
+
+def _act_blocks():
+    out = []
+    for line in open(os.path.join(GOLDEN, "act_quant_blocks.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        x, q, d = [p.split() for p in line.split("|")]
+        out.append((np.array([float(v) for v in x], np.float32), [int(v) for v in q], int(d[0], 16)))
+    return out
+
+
+def test_act_quant_hand_blocks():
+    blocks = _act_blocks()
+    x = np.stack([b[0] for b in blocks]).reshape(1, -1)
+    q, d, _ = oracle.quantize_act(x)
+    for i, (_, qq, dd) in enumerate(blocks):
+        assert q[0, 32 * i:32 * (i + 1)].tolist() == qq
+        assert int(d[0, i]) == dd
+
+
+def test_act_quant_invariants():
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal((4, 4864)) * np.exp(rng.uniform(-30, 30, (4, 1)))).astype(np.float32)
+    x[1, :64] = 0
+    x[2, 100] = -np.float32(3.0e38)
+    q, d, d32 = oracle.quantize_act(x)
+    xb = x.reshape(4, -1, 32).astype(np.float64)
+    qb = q.reshape(4, -1, 32).astype(np.float64)
+    amax = np.abs(xb).max(axis=2)
+    assert np.array_equal(d32, (amax.astype(np.float32) / np.float32(127)))
+    dd = d32.astype(np.float64)[..., None]
+    assert np.all(np.abs(xb - dd * qb) <= dd / 2 * (1 + 2.0 ** -20) + (dd == 0))
+    assert np.all((np.sign(qb) == np.sign(xb)) | (qb == 0))
+    assert np.all(np.abs(qb) <= 127)
+    assert np.all(np.abs(qb).max(axis=2)[amax > 0] == 127)
+    assert np.all(qb[1, :2] == 0) and np.all(d[1, :2] == 0)
+    with np.errstate(over="ignore"):
+        assert np.array_equal(d, d32.astype(np.float16).view(np.uint16))
+
+
+# --------------------------------------------------------------------------
+# P7: integer block dots
+# --------------------------------------------------------------------------
+
+def test_int_dots_closed_forms():
+    K = 64
+    qw = np.full((2, K), 127, np.int8)
+    qw[1, ::2] = -127
+    g = q8gen.assemble_gguf(qw, np.full((2, 2), 0x3C00, np.uint16))
+    xq = np.full((1, K), 127, np.int8)
+    xd = np.full((1, 2), 0x3C00, np.uint16)
+    dots, y, _ = oracle.q8q8(g, xq, xd, 2, K)
+    assert dots[0, 0].tolist() == [516128, 516128]
+    assert dots[0, 1].tolist() == [0, 0]
+    assert y[0].tolist() == [2 * 516128.0, 0.0]
+
+
+# --------------------------------------------------------------------------
+# P8: router
+# --------------------------------------------------------------------------
+
+def test_router_closed_forms():
+    E = 60
+    idx, w = oracle.route(np.zeros((1, E), np.float32), 4)
+    assert idx[0].tolist() == [0, 1, 2, 3]
+    assert np.allclose(w[0], 1 / 60, rtol=1e-15, atol=0)
+    ramp = np.arange(E, dtype=np.float32).reshape(1, E)
+    idx, w = oracle.route(ramp, 4)
+    assert idx[0].tolist() == [59, 58, 57, 56]
+    # softmax of a ramp: p_e = e^e / sum_j e^j, a geometric series
+    z = sum(math.exp(j - 59) for j in range(E))
+    assert np.allclose(w[0], [math.exp(e - 59) / z for e in (59, 58, 57, 56)], rtol=1e-14)
+    # ties: equal top values resolve to the lower index, in order
+    l = np.full((1, E), -1.0, np.float32)
+    l[0, [7, 3, 40, 12, 5]] = 2.0
+    idx, _ = oracle.route(l, 4)
+    assert idx[0].tolist() == [3, 5, 7, 12]
+    # probabilities of all E experts sum to one: with k = E
+    lg = q8gen.logits(3, 5, E)
+    idx, w = oracle.route(lg, E)
+    assert np.allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+    assert all(sorted(r) == list(range(E)) for r in idx.tolist())
+    # descending order of the logits
+    for t in range(5):
+        assert np.all(np.diff(lg[t, idx[t]]) <= 0)
+    # renormalised weights sum to one over the picks
+    _, wr = oracle.route(lg, 4, renormalize=True)
+    assert np.allclose(wr.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# P9: SwiGLU closed forms
+# --------------------------------------------------------------------------
+
+def _unit_matrix(q_rows):
+    q = np.array(q_rows, np.int8)
+    return q8gen.assemble_gguf(q, np.full((q.shape[0], q.shape[1] // 32), 0x3C00, np.uint16))
+
+
+def test_swiglu_closed_forms():
+    K = 32
+    # gate row picks x0, up row picks x1
+    qg = np.zeros((1, K), np.int8); qg[0, 0] = 1
+    qu = np.zeros((1, K), np.int8); qu[0, 1] = 1
+    g8 = _unit_matrix(np.concatenate([qg, qu]))
+    ln3 = np.float32(math.log(3.0))
+    x = np.zeros((3, K), np.float32)
+    x[0, :2] = [0.0, 5.0]     # g = 0            -> h = 0
+    x[1, :2] = [ln3, 4.0]     # sigmoid(ln 3) = 3/4 -> h = 0.75 * ln3 * 4
+    x[2, :2] = [-ln3, 4.0]    # silu(-g) = silu(g) - g
+    out = oracle.gate_up_swiglu(g8, x, 1, K)
+    h = out["h"][:, 0]
+    assert h[0] == 0.0
+    g = float(ln3)
+    assert abs(h[1] - 3.0 * g) <= 4 * 1e-7  # sigmoid(fp32(ln3)) = 3/4 + O(1e-8)
+    assert abs(h[2] - (h[1] - 4 * g)) <= 1e-12
+    # large gate: silu(g) ~ g;  very negative gate: ~ 0
+    x2 = np.zeros((2, K), np.float32)
+    x2[0, :2] = [40.0, 1.5]
+    x2[1, :2] = [-40.0, 1.5]
+    h2 = oracle.gate_up_swiglu(g8, x2, 1, K)["h"][:, 0]
+    assert abs(h2[0] - 60.0) <= 60.0 * 1e-15
+    assert abs(h2[1]) <= 1e-15
+
+
+# --------------------------------------------------------------------------
+# P10: the MoE block reduces to the dense SwiGLU MLP
+# --------------------------------------------------------------------------
+
+def test_moe_reduces_to_dense():
+    H, I = 64, 96
+    gu, _ = q8gen.q8_matrix(41, 2 * I, H)
+    dn, _ = q8gen.q8_matrix(42, H, I)
+    x = q8gen.activations(43, 2, H)
+    idx = np.zeros((2, 1), np.int32)
+    w = np.ones((2, 1), np.float64)
+    y, bound, slot = oracle.moe(gu, dn, None, None, idx, w, x, H, I, 0)
+    # dense MLP: h = SwiGLU(gate_up x), then down h, with h exact in fp64
+    h = oracle.gate_up_swiglu(gu, x, I, H)["h"]
+    q, dbits = q8gen.split_gguf(dn, H, I)
+    wd = q.astype(np.float64) * np.repeat(dbits.view(np.float16).astype(np.float64), 32, axis=1)
+    dense = h @ wd.T
+    assert np.allclose(y, dense, rtol=1e-12, atol=1e-12 * np.abs(h).max())
+    assert np.array_equal(slot[:, 0], y)
+    assert np.all(bound > 0)
+    # a shared expert is added with weight one
+    y2, _, _ = oracle.moe(gu, dn, gu, dn, idx, w, x, H, I, I)
+    assert np.allclose(y2, 2 * y, rtol=1e-12, atol=1e-12 * np.abs(y).max())
+    # two slots on the same expert with weights a, b scale its output by a + b
+    idx2 = np.zeros((2, 2), np.int32)
+    w2 = np.array([[0.25, 0.5], [0.125, 1.0]])
+    gu2 = np.concatenate([gu, gu])  # E = 2 identical experts
+    dn2 = np.concatenate([dn, dn])
+    y3, _, _ = oracle.moe(gu2, dn2, None, None, idx2 + np.array([[0, 1]]), w2, x, H, I, 0)
+    assert np.allclose(y3, y * w2.sum(axis=1)[:, None], rtol=1e-12, atol=1e-12 * np.abs(y).max())
