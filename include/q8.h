@@ -1,0 +1,231 @@
+/*
+ * q8.h -- C ABI of libq8: decode-time products of GGUF Q8_0 block-quantised
+ * weights with activations, for NVIDIA B200 (sm_100a).
+ *
+ * A Q8_0 block holds 32 int8 values q and one binary16 scale d; the weight is
+ * d*q.  The product this library serves is the one the Qwen inference pages
+ * keep returning to: "Lumen v0.3.0 -- profile, parallelize, 4x faster than
+ * v0.2.0" (Phase 7.E.0) measures gate_up, lm_head and down matmuls at most of
+ * a decode step, and "skuznetsov/cogni-ml" README ("Build Qwen CLIs") runs a
+ * Q8_0 GEMV straight over the GGUF block layout.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Shapes: M output rows, K reduction length (a multiple of 32), N activation
+ *    columns (tokens, 1..16).  Activations x are [N][K] fp32 row-major (one
+ *    token per row); outputs are [N][M] fp32 row-major.
+ *  - Memory: every pointer argument is DEVICE memory owned by the caller,
+ *    16-byte aligned.  The library allocates, frees and synchronises nothing in
+ *    these calls; scratch, where a call needs it, is passed in by the caller
+ *    and sized by the matching *_bytes query.
+ *  - Streams: work is enqueued on `stream` (0 = the legacy default stream) and
+ *    returns immediately; results are ready when the stream reaches them.  The
+ *    launches use programmatic dependent launch: a kernel may start streaming
+ *    its weights while the previous kernel on the stream finishes, and reads
+ *    its activations only after that kernel has completed.
+ *  - Errors: arguments are checked on the host before anything is enqueued.
+ *    A rejected call returns a non-zero q8_status and enqueues nothing.  A
+ *    failed launch returns Q8_ERR_CUDA (q8_last_cuda_error() names it).
+ *    Kernels bound every internal wait; a wait that runs out sets a sticky
+ *    device error word that q8_read_device_error() returns.
+ *  - Device data that the host cannot see (expert indices, activation
+ *    values) is trusted: out-of-range expert indices and NaN router logits are
+ *    undefined behaviour, as in "fusedtok 1.3.0" ("Roadmap", 1.2.1: host-side
+ *    validation with a documented device-tensor trust boundary).
+ *
+ * Packed weight layout (what q8_pack_weights writes)
+ * --------------------------------------------------
+ * Rows are taken in groups of 8 (the last group is padded with zero rows).
+ * With B = K/32 blocks per row, group g occupies 272*B bytes at offset
+ * g*272*B:
+ *    q part, 256*B bytes: for each 16-byte column c in [0, 2B) (half a block)
+ *        and each row r in [0, 8): the 16 values q[8g+r][16c .. 16c+15],
+ *        each stored as the byte (q + 128), i.e. q XOR 0x80;
+ *    d part, 16*B bytes: for each block b and row r: the binary16 d[8g+r][b].
+ * Every 16-byte piece is aligned, each (group, column) piece is one 8-row x
+ * 16-byte core matrix of the tensor cores' K-major operand layout, and the
+ * size is exactly 34 bytes per 32 weights (plus the zero rows of the last
+ * group).  q8_unpack_weights restores the GGUF bytes exactly.
+ */
+#ifndef Q8_H_
+#define Q8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st *q8_stream_t;
+
+typedef enum q8_status {
+    Q8_OK = 0,
+    Q8_ERR_INVALID = 1,      /* null pointer or bad enum / flag                 */
+    Q8_ERR_SHAPE = 2,        /* non-positive size, K % 32 != 0, size mismatch   */
+    Q8_ERR_ALIGN = 3,        /* pointer not 16-byte aligned                     */
+    Q8_ERR_NOT_DEVICE = 4,   /* pointer is not device memory                    */
+    Q8_ERR_UNSUPPORTED = 5,  /* legal but outside what the kernels serve (N>16) */
+    Q8_ERR_CUDA = 6,         /* a CUDA call or launch failed                    */
+    Q8_ERR_DEVICE_TIMEOUT = 7 /* a kernel's bounded wait ran out (see below)    */
+} q8_status;
+
+/* Static text for a status code. */
+const char *q8_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread inside the library
+ * ("no error" when none). */
+const char *q8_last_cuda_error(void);
+
+/* Synchronises the current device, then returns and clears the sticky device
+ * error word of the current device: Q8_OK when no kernel recorded a problem,
+ * Q8_ERR_DEVICE_TIMEOUT when some kernel's bounded wait ran out (the kernel
+ * then returned early and its outputs are incomplete).  *detail (nullable)
+ * receives the raw word. */
+q8_status q8_read_device_error(uint32_t *detail);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int q8_version(void);
+
+/* ---------------------------------------------------------------------- */
+/* S1  Weight packer                                                       */
+/* ---------------------------------------------------------------------- */
+
+/* Bytes of the packed layout for an M x K matrix: ceil(M/8) * 8.5 * K.
+ * Returns 0 for invalid shapes (M <= 0, K <= 0, K % 32 != 0). */
+size_t q8_packed_bytes(int64_t M, int64_t K);
+
+/* Re-lay GGUF Q8_0 blocks into the packed layout above.
+ * gguf_blocks: device, M*K/32*34 bytes, row-major blocks [M][K/32], each block
+ *   34 bytes = little-endian binary16 d, then 32 int8 q (the raw GGUF Q8_0
+ *   layout the "skuznetsov/cogni-ml" Q8_0 GEMV probe reads, "Build Qwen CLIs").
+ *   Any byte alignment.
+ * packed: device, q8_packed_bytes(M, K) bytes, 16-byte aligned; fully written.
+ * Pure re-layout: bit-exact and invertible.  One-time cost, not a hot call. */
+q8_status q8_pack_weights(const void *gguf_blocks, int64_t M, int64_t K, void *packed,
+                          q8_stream_t stream);
+
+/* Inverse of q8_pack_weights (test aid): packed -> GGUF bytes [M][K/32][34]. */
+q8_status q8_unpack_weights(const void *packed, int64_t M, int64_t K, void *gguf_blocks,
+                            q8_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* S2/S3  Q8_0 GEMV (N = 1) and small-batch GEMM (N = 2..16), fp32 x       */
+/* ---------------------------------------------------------------------- */
+
+/* y[n][m] = sum_k d[m][k/32] * q[m][k] * x[n][k]   for n < N, m < M.
+ * W: packed (q8_pack_weights) M x K.  x: [N][K] fp32.  y: [N][M] fp32, fully
+ * overwritten.  fp32 arithmetic; each output is within 1e-5 * sum_k |w x| of
+ * the exact value.  The Q8 N=1 decode product of "Lumen v0.3.0" (Phase 7.G)
+ * and the "skuznetsov/cogni-ml" cuda_q8_gemv_probe ("Build Qwen CLIs"),
+ * extended to N <= 16 columns.  N > 16 -> Q8_ERR_UNSUPPORTED. */
+q8_status q8_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                  q8_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* S4  Fused gate_up + SwiGLU                                              */
+/* ---------------------------------------------------------------------- */
+
+/* h[n][i] = silu(g) * u,  g = (W x)[n][i],  u = (W x)[n][I + i],
+ * silu(g) = g / (1 + exp(-g)).  W: packed [2I][K] with the gate rows first
+ * and the up rows after them (the concatenation of the ffn_gate and ffn_up
+ * projections of the "skuznetsov/cogni-ml" FFN probe, "Build Qwen CLIs"; the
+ * SwiGLU MLP of the "augur" README, "Features").  I must be a multiple of 8.
+ * x: [N][K] fp32.  h: [N][I] fp32, fully overwritten.  One launch; g and u
+ * never leave the chip. */
+q8_status q8_gate_up_swiglu(const void *W, const float *x, float *h, int64_t I, int64_t K,
+                            int64_t N, q8_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* S5  MoE router                                                          */
+/* ---------------------------------------------------------------------- */
+
+/* For each token t < T: p = softmax(logits[t][0..E)); idx[t][0..top_k) = the
+ * top_k experts by logit value in descending order, ties to the lowest expert
+ * index ("fusedtok 1.3.0", "API stability"); w[t][j] = p[idx[t][j]], divided
+ * by the sum of the picked p when renormalize != 0.  The router + top-k
+ * expert step of "Add Qwen1.5-MoE Q8_0 CPU and single-token TornadoVM GPU
+ * inference - #144" (PR summary).
+ * logits: [T][E] fp32.  idx: [T][top_k] int32.  w: [T][top_k] fp32.
+ * Limits: 1 <= T <= 16, 1 <= top_k <= min(E, 8), E <= 256. */
+q8_status q8_moe_route(const float *logits, int64_t T, int64_t E, int64_t top_k,
+                       int renormalize, int32_t *idx, float *w, q8_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* S6  Grouped MoE GEMV over the routed experts                            */
+/* ---------------------------------------------------------------------- */
+
+/* Scratch bytes q8_moe_gemv needs for these sizes. */
+size_t q8_moe_workspace_bytes(int64_t T, int64_t E, int64_t top_k, int64_t H, int64_t I,
+                              int64_t I_shared);
+
+/* y[t] = sum_{s < top_k} w[t][s] * Down_e(SwiGLU(GateUp_e x[t]))  (e = idx[t][s])
+ *        + Down_sh(SwiGLU(GateUp_sh x[t]))             (when a shared expert is given)
+ * in two launches: one computes SwiGLU(gate_up) for every selected
+ * (expert, token) pair and the shared expert, the other the down projections
+ * and the weighted sum.  Each launch walks only the selected experts, and an
+ * expert picked by several tokens streams its weights once.  The slot
+ * weighting and shared expert follow the router + top-k expert +
+ * shared-expert FFN block of "Add Qwen1.5-MoE Q8_0 ... - #144" (PR summary);
+ * folding the per-slot launches into one grid follows the routed-expert
+ * launch fusion in that PR's conversation.  The sum over slots runs in slot
+ * order for every output, so results are bit-identical from run to run.
+ *   gate_up_experts: E consecutive packed matrices [2I][H], each
+ *       q8_packed_bytes(2I, H) bytes (gate rows first, as q8_gate_up_swiglu).
+ *   down_experts:    E consecutive packed matrices [H][I], each
+ *       q8_packed_bytes(H, I) bytes.
+ *   shared_gate_up / shared_down: packed [2*I_shared][H] / [H][I_shared], or
+ *       both NULL (with I_shared = 0) for no shared expert.
+ *   idx, w: [T][top_k] as written by q8_moe_route (trusted device data).
+ *   x: [T][H] fp32.  y: [T][H] fp32, fully overwritten.
+ *   workspace: >= q8_moe_workspace_bytes(...) bytes of device scratch, 16-byte
+ *       aligned; its contents on entry do not matter.
+ * Limits: 1 <= T <= 16, top_k <= 8, E <= 256, H, I, I_shared multiples of 32,
+ * I and I_shared multiples of 8. */
+q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
+                      const void *shared_gate_up, const void *shared_down,
+                      const int32_t *idx, const float *w, const float *x, float *y, int64_t T,
+                      int64_t E, int64_t top_k, int64_t H, int64_t I, int64_t I_shared,
+                      void *workspace, size_t workspace_bytes, q8_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* S7  Activation quantisation to Q8_0                                     */
+/* ---------------------------------------------------------------------- */
+
+/* Per 32-block of each row of x: amax = max |x|, d32 = amax / 127 (IEEE fp32
+ * division), q = round-half-away-from-zero(x / d32) (IEEE fp32 division),
+ * clamped to [-127, 127]; amax == 0 gives d = 0 and q = 0; xd = binary16 of
+ * d32, round to nearest even.  Bit-exact.  The per-block int8 quantisation of
+ * fp32 activations in "Add Qwen1.5-MoE Q8_0 ... - #144" ("Key implementation
+ * notes").
+ * x: [N][K] fp32.  xq: [N][K] int8.  xd: [N][K/32] binary16 bits. */
+q8_status q8_quantize_act(const float *x, int8_t *xq, uint16_t *xd, int64_t N, int64_t K,
+                          q8_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* S8  Q8_0 x Q8_0 integer product                                         */
+/* ---------------------------------------------------------------------- */
+
+/* y[n][m] = sum_b d_w[m][b] * d_x[n][b] * dot[n][m][b],
+ * dot[n][m][b] = sum_{i<32} q_w[m][32b+i] * xq[n][32b+i]  (exact int32).
+ * The int8 x int8 accumulation with the Q8_0 scales of "Add Qwen1.5-MoE Q8_0
+ * ... - #144" ("Key implementation notes"), the Q8-native integer dot named
+ * as the next step in "Lumen v0.3.0" ("v0.3 -> v0.4 candidate moves").
+ * N < 16 runs on the integer dot-product units; N == 16 runs on the tensor
+ * cores (tcgen05 int8 MMA, 128 x 16 x 32 per block).
+ * W: packed M x K.  xq, xd: as written by q8_quantize_act.  y: [N][M] fp32.
+ * fp32 result within 1e-5 * sum_b |d_w d_x| sum_i |q_w q_x| of the exact. */
+q8_status q8q8_gemv(const void *W, const int8_t *xq, const uint16_t *xd, float *y, int64_t M,
+                    int64_t K, int64_t N, q8_stream_t stream);
+
+/* Test aid: the int32 block dots themselves, dots[n][m][b] (layout
+ * [N][M][K/32]); bit-exact. */
+q8_status q8q8_block_dots(const void *W, const int8_t *xq, int32_t *dots, int64_t M, int64_t K,
+                          int64_t N, q8_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q8_H_ */

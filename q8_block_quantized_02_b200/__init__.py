@@ -1,0 +1,177 @@
+"""Python binding of libq8 (include/q8.h): Q8_0 decode products on B200.
+
+Argument marshalling only.  Each function forwards to the C entry point of
+the same name: torch CUDA tensors are passed by ``data_ptr()`` (plain integer
+device addresses are accepted too), ``stream`` defaults to torch's current
+stream, and a non-zero status raises :class:`Q8Error`.  Every step of the
+computation runs in the CUDA library; there is no fallback path.  If
+``libq8.so`` is missing or cannot be loaded, every call raises.
+
+Build the library with ``python -m q8_block_quantized_02_b200.build`` (or
+``__graft_entry__.build()``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "Q8Error", "lib_path", "q8_status_string", "q8_last_cuda_error", "q8_read_device_error",
+    "q8_version", "q8_packed_bytes", "q8_pack_weights", "q8_unpack_weights", "q8_gemv",
+    "q8_gate_up_swiglu", "q8_moe_route", "q8_moe_workspace_bytes", "q8_moe_gemv",
+    "q8_quantize_act", "q8q8_gemv", "q8q8_block_dots",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lock = threading.Lock()
+_lib = None
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/q8.h
+_SIGS = {
+    "q8_status_string": (ctypes.c_char_p, [_INT]),
+    "q8_last_cuda_error": (ctypes.c_char_p, []),
+    "q8_read_device_error": (_INT, [ctypes.POINTER(ctypes.c_uint32)]),
+    "q8_version": (_INT, []),
+    "q8_packed_bytes": (_SZ, [_I64, _I64]),
+    "q8_pack_weights": (_INT, [_P, _I64, _I64, _P, _P]),
+    "q8_unpack_weights": (_INT, [_P, _I64, _I64, _P, _P]),
+    "q8_gemv": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
+    "q8_gate_up_swiglu": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
+    "q8_moe_route": (_INT, [_P, _I64, _I64, _I64, _INT, _P, _P, _P]),
+    "q8_moe_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64, _I64, _I64]),
+    "q8_moe_gemv": (_INT, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64,
+                           _P, _SZ, _P]),
+    "q8_quantize_act": (_INT, [_P, _P, _P, _I64, _I64, _P]),
+    "q8q8_gemv": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "q8q8_block_dots": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
+}
+
+
+class Q8Error(RuntimeError):
+    """A libq8 call returned a non-zero q8_status."""
+
+    def __init__(self, func: str, status: int):
+        lib = _load()
+        text = lib.q8_status_string(status).decode()
+        detail = lib.q8_last_cuda_error().decode() if status == 6 else ""
+        super().__init__(f"{func}: {text}" + (f" [{detail}]" if detail else ""))
+        self.status = status
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, "libq8.so")
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            path = lib_path()
+            if not os.path.exists(path):
+                raise RuntimeError(f"libq8.so is not built ({path}); run "
+                                   "`python -m q8_block_quantized_02_b200.build`")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in _SIGS.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _call(name, *args):
+    st = getattr(_load(), name)(*args)
+    if st != 0:
+        raise Q8Error(name, st)
+
+
+def q8_status_string(status: int) -> str:
+    return _load().q8_status_string(int(status)).decode()
+
+
+def q8_last_cuda_error() -> str:
+    return _load().q8_last_cuda_error().decode()
+
+
+def q8_read_device_error():
+    """Synchronise the device; return (status, raw word) and clear the word."""
+    w = ctypes.c_uint32(0)
+    st = _load().q8_read_device_error(ctypes.byref(w))
+    return st, w.value
+
+
+def q8_version() -> int:
+    return _load().q8_version()
+
+
+def q8_packed_bytes(M: int, K: int) -> int:
+    return int(_load().q8_packed_bytes(M, K))
+
+
+def q8_pack_weights(gguf_blocks, M, K, packed, stream=None):
+    _call("q8_pack_weights", _ptr(gguf_blocks), M, K, _ptr(packed), _stream(stream))
+
+
+def q8_unpack_weights(packed, M, K, gguf_blocks, stream=None):
+    _call("q8_unpack_weights", _ptr(packed), M, K, _ptr(gguf_blocks), _stream(stream))
+
+
+def q8_gemv(W, x, y, M, K, N, stream=None):
+    _call("q8_gemv", _ptr(W), _ptr(x), _ptr(y), M, K, N, _stream(stream))
+
+
+def q8_gate_up_swiglu(W, x, h, I, K, N, stream=None):
+    _call("q8_gate_up_swiglu", _ptr(W), _ptr(x), _ptr(h), I, K, N, _stream(stream))
+
+
+def q8_moe_route(logits, T, E, top_k, renormalize, idx, w, stream=None):
+    _call("q8_moe_route", _ptr(logits), T, E, top_k, int(bool(renormalize)), _ptr(idx), _ptr(w),
+          _stream(stream))
+
+
+def q8_moe_workspace_bytes(T, E, top_k, H, I, I_shared) -> int:
+    return int(_load().q8_moe_workspace_bytes(T, E, top_k, H, I, I_shared))
+
+
+def q8_moe_gemv(gate_up_experts, down_experts, shared_gate_up, shared_down, idx, w, x, y, T, E,
+                top_k, H, I, I_shared, workspace, workspace_bytes, stream=None):
+    _call("q8_moe_gemv", _ptr(gate_up_experts), _ptr(down_experts), _ptr(shared_gate_up),
+          _ptr(shared_down), _ptr(idx), _ptr(w), _ptr(x), _ptr(y), T, E, top_k, H, I, I_shared,
+          _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def q8_quantize_act(x, xq, xd, N, K, stream=None):
+    _call("q8_quantize_act", _ptr(x), _ptr(xq), _ptr(xd), N, K, _stream(stream))
+
+
+def q8q8_gemv(W, xq, xd, y, M, K, N, stream=None):
+    _call("q8q8_gemv", _ptr(W), _ptr(xq), _ptr(xd), _ptr(y), M, K, N, _stream(stream))
+
+
+def q8q8_block_dots(W, xq, dots, M, K, N, stream=None):
+    _call("q8q8_block_dots", _ptr(W), _ptr(xq), _ptr(dots), M, K, N, _stream(stream))

@@ -1,0 +1,91 @@
+// q8q8.cuh -- S7: activation quantisation to Q8_0, and the bit-exact int32
+// block-dot test aid of S8.  (The Q8 x Q8 products themselves run in the tile
+// kernel's kModeQ8Q8 and in the tensor-core kernel.)
+#pragma once
+
+#include "q8_device.cuh"
+
+namespace q8 {
+
+// One thread per (row n, block b): amax over the block, d32 = amax / 127,
+// q = roundf(x / d32) clamped to +-127 (roundf rounds half away from zero),
+// stored scale = binary16 RN of d32.  Divisions are IEEE round-to-nearest
+// (__fdiv_rn) so the result is bit-exact with any IEEE implementation of the
+// same steps.
+__global__ void quantize_act_kernel(const float *__restrict__ x, int8_t *__restrict__ xq,
+                                    uint16_t *__restrict__ xd, int64_t N, int64_t K) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t B = K / 32;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N * B;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 *src = reinterpret_cast<const float4 *>(x + i * 32);
+        float v[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float4 f = src[k];
+            v[4 * k] = f.x;
+            v[4 * k + 1] = f.y;
+            v[4 * k + 2] = f.z;
+            v[4 * k + 3] = f.w;
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float a = fabsf(v[k]);
+            if (a > amax) amax = a;
+        }
+        const float d32 = __fdiv_rn(amax, 127.0f);
+        uint32_t packed[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                int q = 0;
+                if (d32 != 0.0f) {
+                    float r = roundf(__fdiv_rn(v[4 * k + b], d32));
+                    r = fminf(fmaxf(r, -127.0f), 127.0f);
+                    q = (int)r;
+                }
+                word |= ((uint32_t)(q & 0xff)) << (8 * b);
+            }
+            packed[k] = word;
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(xq + i * 32);
+        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        xd[i] = __half_as_ushort(__float2half_rn(d32));
+    }
+}
+
+// Test aid: dots[n][m][b] = sum_i q_w[m][32b+i] * xq[n][32b+i], one thread per
+// output, straight from the packed layout.
+__global__ void block_dots_kernel(const uint8_t *__restrict__ W, const int8_t *__restrict__ xq,
+                                  int32_t *__restrict__ dots, int64_t M, int64_t K, int64_t N) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t B = K / 32;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N * M * B;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t b = i % B, m = (i / B) % M, n = i / (B * M);
+        const uint8_t *grp = W + (m / kGroupRows) * kGroupBytesPerBlock * B;
+        const int r = (int)(m % kGroupRows);
+        const uint4 lo = *reinterpret_cast<const uint4 *>(grp + (2 * b) * kColBytes + r * 16);
+        const uint4 hi = *reinterpret_cast<const uint4 *>(grp + (2 * b + 1) * kColBytes + r * 16);
+        const uint4 xa = *reinterpret_cast<const uint4 *>(xq + n * K + 32 * b);
+        const uint4 xb = *reinterpret_cast<const uint4 *>(xq + n * K + 32 * b + 16);
+        const uint32_t wq[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        const uint32_t xx[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+        int dot = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            int d;
+            asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(wq[k] ^ 0x80808080u), "r"(xx[k]), "r"(dot));
+            dot = d;
+        }
+        dots[i] = dot;
+    }
+}
+
+}  // namespace q8

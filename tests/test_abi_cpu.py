@@ -1,0 +1,74 @@
+"""CPU-only checks of the C-ABI library: it builds for sm_100a, loads, exports
+every symbol include/q8.h declares, and its pure host queries answer as
+documented.  No compute call is made (there is no GPU here)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import shutil
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "q8.h")
+
+
+def _declared_functions() -> list[str]:
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(q8\w*)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if shutil.which("nvcc") is None and not os.path.exists("/usr/local/cuda/bin/nvcc"):
+        pytest.skip("nvcc not available")
+    from q8_block_quantized_02_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("q8_pack_weights", "q8_gemv", "q8_gate_up_swiglu", "q8_moe_route",
+                     "q8_moe_gemv", "q8_quantize_act", "q8q8_gemv", "q8q8_block_dots",
+                     "q8_packed_bytes", "q8_moe_workspace_bytes", "q8_unpack_weights"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"not exported: {missing}"
+
+
+def test_binding_covers_the_header():
+    import q8_block_quantized_02_b200 as q8
+    for n in _declared_functions():
+        assert hasattr(q8, n), f"python binding lacks {n}"
+
+
+def test_packed_bytes(lib):
+    f = lib.q8_packed_bytes
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    # 34 bytes per 32 weights, rows padded to a multiple of 8
+    assert f(8, 32) == 8 * 34
+    assert f(1152, 896) == 1152 * 896 // 32 * 34
+    assert f(1, 64) == 8 * 2 * 34
+    assert f(151936, 896) == 151936 * 28 * 34
+    assert f(0, 32) == 0 and f(8, 0) == 0 and f(8, 48) == 0 and f(-8, 32) == 0
+
+
+def test_status_strings(lib):
+    f = lib.q8_status_string
+    f.restype = ctypes.c_char_p
+    f.argtypes = [ctypes.c_int]
+    texts = {f(i).decode() for i in range(8)}
+    assert len(texts) == 8 and "ok" in texts
+    assert f(99).decode() == "unknown status"
+
+
+def test_library_targets_sm100a_only():
+    from q8_block_quantized_02_b200 import build
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.NVCC_FLAGS)
