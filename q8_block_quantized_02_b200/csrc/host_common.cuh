@@ -127,11 +127,66 @@ inline EncodeTiledFn encode_tiled_fn() {
     return fn;
 }
 
+// Encoded maps are kept in a small per-thread cache keyed by every encoding
+// input: decode loops call the same matrices with the same buffers again and
+// again, and encoding costs microseconds of host time.
+struct MapKey {
+    const void *base;
+    uint64_t d0, d1, d2, s1, s2;
+    uint32_t b0, b1, b2;
+    int dtype;
+    int stream_l2;
+    int device;
+    bool operator==(const MapKey &o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+
+struct MapEntry {
+    MapKey key;
+    CUtensorMap map;
+    bool valid;
+};
+
+constexpr int kMapCacheSize = 256;
+
+inline q8_status encode_map_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
+                               uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+                               uint32_t b0, uint32_t b1, uint32_t b2, bool stream_l2);
+
 // A 3-D tensor map over `base` with the given extents, byte strides of dims 1
 // and 2, and box; zero fill outside the tensor, no swizzle.
 inline q8_status make_map_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
                              uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
                              uint32_t b0, uint32_t b1, uint32_t b2, bool stream_l2) {
+    static thread_local MapEntry cache[kMapCacheSize];
+    MapKey key;
+    std::memset(&key, 0, sizeof(key));
+    key.base = base;
+    key.d0 = d0; key.d1 = d1; key.d2 = d2; key.s1 = s1; key.s2 = s2;
+    key.b0 = b0; key.b1 = b1; key.b2 = b2;
+    key.dtype = (int)dtype;
+    key.stream_l2 = stream_l2 ? 1 : 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    key.device = dev;
+    uint64_t h = reinterpret_cast<uintptr_t>(base) * 0x9E3779B97F4A7C15ull;
+    h ^= (d1 * 31 + d2) * 0xC2B2AE3D27D4EB4Full ^ (b1 * 131 + b2 * 7 + (uint64_t)dtype);
+    MapEntry &e = cache[(h >> 32) % kMapCacheSize];
+    if (e.valid && e.key == key) {
+        *map = e.map;
+        return Q8_OK;
+    }
+    q8_status st = encode_map_3d(map, dtype, base, d0, d1, d2, s1, s2, b0, b1, b2, stream_l2);
+    if (st == Q8_OK) {
+        e.key = key;
+        e.map = *map;
+        e.valid = true;
+    }
+    return st;
+}
+
+inline q8_status encode_map_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
+                               uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+                               uint32_t b0, uint32_t b1, uint32_t b2, bool stream_l2) {
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) {
         snprintf(last_error_buf(), 256, "cuTensorMapEncodeTiled unavailable");

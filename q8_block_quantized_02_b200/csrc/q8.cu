@@ -55,58 +55,56 @@ struct TilePlan {
     size_t smem;
 };
 
-// Choose the tile height (TG groups) and stage width (CS columns) for `units`
-// row groups of C 16-byte columns.  A stage carries about 32 KB of weights;
-// its activation slice is kept at or under 16 KB.  Among the legal shapes the
-// one with the least per-CTA work (waves x tile size) wins, with a small
-// penalty for shapes whose groups are split across warps.
+static int64_t pow2_ceil(int64_t v) {
+    int64_t p = 1;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+// Launch shape for `units` row groups of C 16-byte columns.  The grid is one
+// CTA per SM (or one per unit when there are fewer units); each CTA owns a
+// contiguous unit range, taken in tiles of TG units.  A stage holds about
+// 32 KB of weights (16 KB for each half of a SwiGLU tile) and at most 16 KB of
+// activations.
 static TilePlan plan_tile(int64_t units, int64_t C, int64_t N, int mode, int sms) {
     const bool swiglu = mode == kModeSwiGLU;
-    const int pairs = swiglu ? 128 : 256;
-    const int tg_max = swiglu ? 8 : 16;
-    const int64_t c_pad = round_up(C, 8);
-    const int nb = nmax_for(N);
+    const int64_t grid = units < sms ? units : sms;
+    const int64_t upc = ceil_div(units, grid);
+    const int64_t tg_max = swiglu ? 8 : 16;
+    const int64_t tg = std::min<int64_t>(tg_max, pow2_ceil(upc));
+    const int64_t pairs = swiglu ? 128 : 256;
+    const int64_t eff = std::min<int64_t>(upc, tg);
     const int64_t x_col_bytes = mode == kModeQ8Q8 ? 16 : 64;  // per column per activation row
-    double best_cost = 1e300;
-    int best_tg = 1, best_cs = 8;
-    for (int tg = 1; tg <= tg_max; tg *= 2) {
-        int64_t cs = pairs / tg;
-        if (cs > c_pad) cs = c_pad;
-        while (cs > 8 && nb * cs * x_col_bytes > 16384) cs -= 8;
-        const int64_t tiles = ceil_div(units, tg);
-        const int64_t waves = ceil_div(tiles, sms);
-        const int64_t ksteps = ceil_div(C, cs);
-        double cost = (double)waves * tg * ksteps * cs * (tg < 8 ? 1.15 : 1.0);
-        if (cost < best_cost - 1e-9 || (cost <= best_cost + 1e-9 && tg > best_tg)) {
-            best_cost = cost;
-            best_tg = tg;
-            best_cs = (int)cs;
-        }
-    }
+    const int nb = nmax_for(N);
+    int64_t cs = std::max<int64_t>(8, (pairs / eff) / 8 * 8);
+    cs = std::min<int64_t>(cs, round_up(C, 8));
+    while (cs > 8 && nb * cs * x_col_bytes > 16384) cs -= 8;
     TilePlan p;
     TileArgs &a = p.a;
     a = TileArgs{};
     a.N = (int)N;
     a.C = (int)C;
-    a.TG = best_tg;
-    a.CS = best_cs;
-    a.ksteps = (int)ceil_div(C, best_cs);
-    a.n_tiles = (int)ceil_div(units, best_tg);
-    const int halves = swiglu ? 2 : 1;
-    a.q_half = (uint32_t)(best_tg * best_cs * kColBytes);
-    const uint32_t d_box = (uint32_t)(best_tg * (best_cs / 2) * 16);
-    a.d_half = (uint32_t)round_up(d_box, 128);
+    a.B = (int)(C / 2);
+    a.units = (int)units;
+    a.TG = (int)tg;
+    a.CS = (int)cs;
+    a.ksteps = (int)ceil_div(C, cs);
+    a.NQ = (int)ceil_div(C, 4);
+    const uint32_t halves = swiglu ? 2 : 1;
+    a.q_box = (uint32_t)(cs * kColBytes);
+    a.d_box = (uint32_t)(cs * 8);
+    a.d_slot = (uint32_t)round_up(a.d_box, 128);
+    a.x_box = (uint32_t)(N * cs * x_col_bytes);
+    a.q_half = (uint32_t)tg * a.q_box;
     a.d_off = halves * a.q_half;
+    a.d_half = (uint32_t)tg * a.d_slot;
     a.x_off = a.d_off + halves * a.d_half;
-    const uint32_t x_box = (uint32_t)(N * best_cs * x_col_bytes);
-    a.stage_bytes = (uint32_t)round_up(a.x_off + x_box, 128);
-    a.tx_bytes = halves * (a.q_half + d_box) + x_box;
+    a.stage_bytes = (uint32_t)round_up(a.x_off + a.x_box, 128);
     int stages = (int)(112 * 1024 / a.stage_bytes);
-    if (stages < 2) stages = 2;
-    if (stages > 6) stages = 6;
-    a.stages = stages;
-    p.grid = (int)(a.n_tiles < sms ? a.n_tiles : sms);
-    p.smem = (size_t)stages * a.stage_bytes + 16 * stages + tile_red_floats(nb) * 4 + 16;
+    a.stages = stages < 2 ? 2 : stages > 8 ? 8 : stages;
+    p.grid = (int)grid;
+    const int sets = swiglu ? 4 : 2;
+    p.smem = (size_t)a.stages * a.stage_bytes + 16 * a.stages + tile_red_floats(nb, sets) * 4 + 16;
     return p;
 }
 
@@ -122,17 +120,16 @@ static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, floa
     TileArgs &a = p.a;
     a.y = y;
     a.xd = xd;
-    a.B = (int)B;
     a.M_out = (int)rows_out;
     a.up_group0 = swiglu ? (int)units : 0;
     if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
     const uint64_t gstride = (uint64_t)kGroupBytesPerBlock * B;
     CUtensorMap tq, td, tx;
     Q8_CHECK(make_map_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, kColBytes, C, total_groups,
-                         kColBytes, gstride, kColBytes, a.CS, a.TG, true));
+                         kColBytes, gstride, kColBytes, a.CS, 1, true));
     Q8_CHECK(make_map_3d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT16,
                          static_cast<const uint8_t *>(W) + 256 * B, 8, B, total_groups, 16, gstride,
-                         8, a.CS / 2, a.TG, true));
+                         8, a.CS / 2, 1, true));
     if (mode == kModeQ8Q8)
         Q8_CHECK(make_map_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, x, 16, C, N, 16, (uint64_t)K, 16,
                              a.CS, (uint32_t)N, false));

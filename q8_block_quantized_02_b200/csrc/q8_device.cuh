@@ -175,6 +175,66 @@ __device__ __forceinline__ void dequant16(const uint4 v, float (&w)[16]) {
     }
 }
 
+// Packed fp32 pairs (sm_100 f32x2 instructions: two IEEE fp32 operations per
+// instruction, each rounded as the scalar one would be).
+__device__ __forceinline__ uint64_t pack_u32x2(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 unpack_f32x2(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return make_float2(lo, hi);
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// Dequantise 16 packed bytes into 8 fp32 pairs (q0,q1), (q2,q3), ...: a byte
+// permute per weight, then one paired subtraction of 2^23 + 128 per two.
+__device__ __forceinline__ void dequant16_x2(const uint4 v, uint64_t (&w)[8]) {
+    const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+    const uint32_t nb = __float_as_uint(-8388736.0f);
+    const uint64_t neg_bias = pack_u32x2(nb, nb);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t b0 = __byte_perm(words[i], 0x4B000000u, 0x7540u);
+        const uint32_t b1 = __byte_perm(words[i], 0x4B000000u, 0x7541u);
+        const uint32_t b2 = __byte_perm(words[i], 0x4B000000u, 0x7542u);
+        const uint32_t b3 = __byte_perm(words[i], 0x4B000000u, 0x7543u);
+        w[2 * i] = add_f32x2(pack_u32x2(b0, b1), neg_bias);
+        w[2 * i + 1] = add_f32x2(pack_u32x2(b2, b3), neg_bias);
+    }
+}
+
+// sum_i w_i x_i over 16 values held as 8 pairs each (two interleaved chains).
+__device__ __forceinline__ float dot16_x2(const uint64_t (&w)[8], const ulonglong2 x0,
+                                          const ulonglong2 x1, const ulonglong2 x2,
+                                          const ulonglong2 x3) {
+    uint64_t a = mul_f32x2(w[0], x0.x), b = mul_f32x2(w[1], x0.y);
+    a = fma_f32x2(w[2], x1.x, a);
+    b = fma_f32x2(w[3], x1.y, b);
+    a = fma_f32x2(w[4], x2.x, a);
+    b = fma_f32x2(w[5], x2.y, b);
+    a = fma_f32x2(w[6], x3.x, a);
+    b = fma_f32x2(w[7], x3.y, b);
+    const float2 s = unpack_f32x2(add_f32x2(a, b));
+    return s.x + s.y;
+}
+
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
 }  // namespace q8
