@@ -242,6 +242,10 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
+    # CUDAGraph.replay() launches on torch's current stream: make it `stream`
+    # for every replay below, so the events bracket exactly those launches.
+    torch.cuda.set_stream(stream)
+
     # ---- warm-up replays ----
     for _ in range(args.warmup):
         graph.replay()
@@ -297,12 +301,11 @@ def run_ours(args):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(e2e_steps):
-            x_dev.copy_(x_host, non_blocking=True)
-            graph.replay()
-            logits_host.copy_(y_bufs[lm], non_blocking=True)
-            stream.synchronize()
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        graph.replay()
+        logits_host.copy_(y_bufs[lm], non_blocking=True)
+        stream.synchronize()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_elapsed = e0.elapsed_time(e1) / 1e3

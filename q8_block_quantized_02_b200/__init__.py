@@ -150,7 +150,7 @@ def q8_gate_up_swiglu(W, x, h, I, K, N, stream=None):
 
 
 def q8_moe_route(logits, T, E, top_k, renormalize, idx, w, stream=None):
-    _call("q8_moe_route", _ptr(logits), T, E, top_k, int(bool(renormalize)), _ptr(idx), _ptr(w),
+    _call("q8_moe_route", _ptr(logits), T, E, top_k, int(renormalize), _ptr(idx), _ptr(w),
           _stream(stream))
 
 

@@ -16,31 +16,73 @@ namespace q8 {
 // ---------------------------------------------------------------------------
 // tile GEMM (S2 / S3 / S4)
 // ---------------------------------------------------------------------------
-using TileKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, TileArgs);
+using TileKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+                           TileArgs);
 
+// `wide` selects the 16-consumer-warp column kernel (N = 1 only): more warps
+// per SM for matrices with many tiles per CTA; the 8-warp kernels leave room
+// for the next kernel on the stream to become resident early.
 template <int MODE>
-static TileKernel tile_kernel_mode(int nmax) {
+static TileKernel tile_kernel_mode(int nmax, bool wide) {
     switch (nmax) {
-        case 1: return &tile_gemm_kernel<1, MODE>;
-        case 2: return &tile_gemm_kernel<2, MODE>;
-        case 4: return &tile_gemm_kernel<4, MODE>;
+        case 1: return wide ? &cols_kernel<1, MODE, 16> : &cols_kernel<1, MODE, 8>;
+        case 2: return &cols_kernel<2, MODE, 8>;
+        case 4: return &cols_kernel<4, MODE, 8>;
         case 8: return &tile_gemm_kernel<8, MODE>;
         default: return &tile_gemm_kernel<16, MODE>;
     }
 }
 
-static TileKernel tile_kernel_for(int nmax, int mode) {
-    return mode == kModeF32 ? tile_kernel_mode<kModeF32>(nmax)
-           : mode == kModeSwiGLU ? tile_kernel_mode<kModeSwiGLU>(nmax)
-                                 : tile_kernel_mode<kModeQ8Q8>(nmax);
+static TileKernel tile_kernel_for(int nmax, int mode, bool wide = false) {
+    return mode == kModeF32 ? tile_kernel_mode<kModeF32>(nmax, wide)
+           : mode == kModeSwiGLU ? tile_kernel_mode<kModeSwiGLU>(nmax, wide)
+                                 : tile_kernel_mode<kModeQ8Q8>(nmax, wide);
+}
+
+// Launch geometry of the kernel serving (nmax, mode): threads per CTA, the
+// column-owner kernel's units per tile (0 for the group-owner kernel) and the
+// floats of its partial-sum area.
+struct KernelShape {
+    int threads, tgm, red_floats;
+};
+
+template <int NMAX, int MODE, int CW>
+static KernelShape cols_shape() {
+    using C = ColsCfg<NMAX, MODE, CW>;
+    return {C::THREADS, C::TGM, C::RED_FLOATS};
+}
+
+static KernelShape kernel_shape(int nmax, int mode, bool wide = false) {
+    if (nmax <= 4) {
+        switch (mode * 8 + nmax) {
+            case kModeF32 * 8 + 1: return wide ? cols_shape<1, kModeF32, 16>() : cols_shape<1, kModeF32, 8>();
+            case kModeF32 * 8 + 2: return cols_shape<2, kModeF32, 8>();
+            case kModeF32 * 8 + 4: return cols_shape<4, kModeF32, 8>();
+            case kModeSwiGLU * 8 + 1:
+                return wide ? cols_shape<1, kModeSwiGLU, 16>() : cols_shape<1, kModeSwiGLU, 8>();
+            case kModeSwiGLU * 8 + 2: return cols_shape<2, kModeSwiGLU, 8>();
+            case kModeSwiGLU * 8 + 4: return cols_shape<4, kModeSwiGLU, 8>();
+            case kModeQ8Q8 * 8 + 1: return wide ? cols_shape<1, kModeQ8Q8, 16>() : cols_shape<1, kModeQ8Q8, 8>();
+            case kModeQ8Q8 * 8 + 2: return cols_shape<2, kModeQ8Q8, 8>();
+            default: return cols_shape<4, kModeQ8Q8, 8>();
+        }
+    }
+    const int sets = mode == kModeSwiGLU ? 4 : 2;
+    return {kTileThreads, 0, tile_red_floats(nmax, sets)};
 }
 
 static cudaError_t setup_tile_kernels(int max_smem) {
     const int nm[5] = {1, 2, 4, 8, 16};
-    for (int i = 0; i < 5; ++i)
+    for (int i = 0; i < 6; ++i)
         for (int mode = 0; mode < 3; ++mode) {
-            cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void *>(tile_kernel_for(nm[i], mode)),
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+            const void *k = reinterpret_cast<const void *>(
+                i < 5 ? tile_kernel_for(nm[i], mode) : tile_kernel_for(1, mode, true));
+            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+            if (e != cudaSuccess) return e;
+            // every tile kernel asks for the largest shared-memory carveout, so
+            // consecutive kernels keep one SM configuration and can co-reside
+            e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared);
             if (e != cudaSuccess) return e;
         }
     return cudaSuccess;
@@ -52,6 +94,8 @@ static int nmax_for(int64_t N) { return N <= 1 ? 1 : N <= 2 ? 2 : N <= 4 ? 4 : N
 struct TilePlan {
     TileArgs a;
     int grid;
+    int threads;
+    bool wide;
     size_t smem;
 };
 
@@ -68,17 +112,25 @@ static int64_t pow2_ceil(int64_t v) {
 // activations.
 static TilePlan plan_tile(int64_t units, int64_t C, int64_t N, int mode, int sms) {
     const bool swiglu = mode == kModeSwiGLU;
+    const int nb = nmax_for(N);
+    const bool cols_path = nb <= 4;  // column-owner kernel (see tile_gemm.cuh)
     const int64_t grid = units < sms ? units : sms;
     const int64_t upc = ceil_div(units, grid);
-    const int64_t tg_max = swiglu ? 8 : 16;
-    const int64_t tg = std::min<int64_t>(tg_max, pow2_ceil(upc));
+    // many tiles per CTA: take the 16-warp kernel (it fills the SM on its own);
+    // otherwise stay within half an SM so the next kernel can co-reside
+    const bool wide = nb == 1 && upc >= 32;
+    const KernelShape ks = kernel_shape(nb, mode, wide);
+    int64_t tg = cols_path ? ks.tgm : std::min<int64_t>(swiglu ? 8 : 16, pow2_ceil(upc));
+    tg = std::min<int64_t>(tg, upc);  // a stage never holds more units than a CTA owns
+    // weight (unit x column) pairs per stage: ~32 KB of packed weights
     const int64_t pairs = swiglu ? 128 : 256;
     const int64_t eff = std::min<int64_t>(upc, tg);
     const int64_t x_col_bytes = mode == kModeQ8Q8 ? 16 : 64;  // per column per activation row
-    const int nb = nmax_for(N);
-    int64_t cs = std::max<int64_t>(8, (pairs / eff) / 8 * 8);
-    cs = std::min<int64_t>(cs, round_up(C, 8));
-    while (cs > 8 && nb * cs * x_col_bytes > 16384) cs -= 8;
+    // CS is a multiple of 16, so every scale box is a multiple of 128 bytes and
+    // a tile box lands in shared memory exactly as TG unit boxes would
+    int64_t cs = std::max<int64_t>(16, (pairs / eff) / 16 * 16);
+    cs = std::min<int64_t>(cs, round_up(C, 16));
+    while (cs > 16 && nb * cs * x_col_bytes > 16384) cs -= 16;
     TilePlan p;
     TileArgs &a = p.a;
     a = TileArgs{};
@@ -93,18 +145,27 @@ static TilePlan plan_tile(int64_t units, int64_t C, int64_t N, int mode, int sms
     const uint32_t halves = swiglu ? 2 : 1;
     a.q_box = (uint32_t)(cs * kColBytes);
     a.d_box = (uint32_t)(cs * 8);
-    a.d_slot = (uint32_t)round_up(a.d_box, 128);
+    a.d_slot = a.d_box;
     a.x_box = (uint32_t)(N * cs * x_col_bytes);
     a.q_half = (uint32_t)tg * a.q_box;
     a.d_off = halves * a.q_half;
     a.d_half = (uint32_t)tg * a.d_slot;
     a.x_off = a.d_off + halves * a.d_half;
     a.stage_bytes = (uint32_t)round_up(a.x_off + a.x_box, 128);
-    int stages = (int)(112 * 1024 / a.stage_bytes);
-    a.stages = stages < 2 ? 2 : stages > 8 ? 8 : stages;
+    const int64_t fixed = (cols_path ? 32 : 0) + (int64_t)ks.red_floats * 4 + 16;
+    const int64_t budget = (wide ? 124 * 1024 : 100 * 1024) - fixed;
+    int64_t stages = budget / a.stage_bytes;
+    stages = stages < 2 ? 2 : stages > 8 ? 8 : stages;
+    // no more buffers than a CTA ever fills: small kernels then leave room for
+    // the next kernel on the stream to become resident early
+    stages = std::min<int64_t>(stages, ceil_div(upc, tg) * a.ksteps);
+    a.stages = (int)stages;
     p.grid = (int)grid;
-    const int sets = swiglu ? 4 : 2;
-    p.smem = (size_t)a.stages * a.stage_bytes + 16 * a.stages + tile_red_floats(nb, sets) * 4 + 16;
+    p.threads = ks.threads;
+    p.wide = wide;
+    // must match the kernels' shared-memory carve-up (tile_gemm.cuh)
+    p.smem = (size_t)a.stages * a.stage_bytes + 16 * a.stages + (cols_path ? 32 : 0) +
+             (size_t)ks.red_floats * 4 + 16;
     return p;
 }
 
@@ -124,23 +185,29 @@ static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, floa
     a.up_group0 = swiglu ? (int)units : 0;
     if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
     const uint64_t gstride = (uint64_t)kGroupBytesPerBlock * B;
-    CUtensorMap tq, td, tx;
+    if ((uint64_t)units * (uint64_t)p.grid >= (1ull << 31)) return Q8_ERR_UNSUPPORTED;
+    CUtensorMap tq, td, tq1, td1, tx;
+    const uint8_t *dbase = static_cast<const uint8_t *>(W) + 256 * B;
     Q8_CHECK(make_map_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, kColBytes, C, total_groups,
+                         kColBytes, gstride, kColBytes, a.CS, a.TG, true));
+    Q8_CHECK(make_map_3d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT16, dbase, 8, B, total_groups, 16,
+                         gstride, 8, a.CS / 2, a.TG, true));
+    Q8_CHECK(make_map_3d(&tq1, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, kColBytes, C, total_groups,
                          kColBytes, gstride, kColBytes, a.CS, 1, true));
-    Q8_CHECK(make_map_3d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT16,
-                         static_cast<const uint8_t *>(W) + 256 * B, 8, B, total_groups, 16, gstride,
-                         8, a.CS / 2, 1, true));
+    Q8_CHECK(make_map_3d(&td1, CU_TENSOR_MAP_DATA_TYPE_UINT16, dbase, 8, B, total_groups, 16,
+                         gstride, 8, a.CS / 2, 1, true));
     if (mode == kModeQ8Q8)
         Q8_CHECK(make_map_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, x, 16, C, N, 16, (uint64_t)K, 16,
                              a.CS, (uint32_t)N, false));
     else
         Q8_CHECK(make_map_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, C, N, 64,
                              (uint64_t)K * 4, 16, a.CS, (uint32_t)N, false));
-    TileKernel k = tile_kernel_for(nmax_for(N), mode);
+    TileKernel k = tile_kernel_for(nmax_for(N), mode, p.wide);
     const char *name = mode == kModeF32      ? "q8_gemv launch"
                        : mode == kModeSwiGLU ? "q8_gate_up_swiglu launch"
                                              : "q8q8_gemv launch";
-    return launch_pdl(k, dim3(p.grid), dim3(kTileThreads), p.smem, stream, name, tq, td, tx, a);
+    return launch_pdl(k, dim3(p.grid), dim3(p.threads), p.smem, stream, name, tq, td, tq1, td1,
+                      tx, a);
 }
 
 }  // namespace q8

@@ -56,7 +56,7 @@ struct TileArgs {
     int stages;          // ring depth
     uint32_t q_box;      // bytes of one unit's q box (CS * 128)
     uint32_t d_box;      // bytes of one unit's scale box (CS * 8)
-    uint32_t d_slot;     // shared-memory stride of scale boxes (128-aligned)
+    uint32_t d_slot;     // shared-memory stride of unit scale boxes (= d_box)
     uint32_t x_box;      // bytes of the activation box
     uint32_t q_half;     // TG * q_box
     uint32_t d_off;      // offset of the scale region
@@ -173,24 +173,195 @@ __device__ __forceinline__ void store_unit(const TileArgs &a, int unit, int r, c
             a.y[(size_t)n * a.M_out + row] = MODE == kModeSwiGLU ? silu_mul(v0[n], v1[n]) : v0[n];
 }
 
-template <int NMAX, int MODE>
-__global__ void __launch_bounds__(kTileThreads, 1)
-    tile_gemm_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap td,
-                     const __grid_constant__ CUtensorMap tx, const TileArgs a) {
-    constexpr int SETS = tile_acc_sets<MODE>();
+// ---------------------------------------------------------------------------
+// producer: one elected thread streams the tiles' TMA boxes into the ring
+// ---------------------------------------------------------------------------
+template <int MODE>
+__device__ __forceinline__ void tile_produce(uint8_t *smem, uint32_t full0, uint32_t empty0,
+                                             volatile int *abort_flag, volatile int *issued,
+                                             const TileArgs &a, int u0, int u1, int total,
+                                             const CUtensorMap *tq, const CUtensorMap *td,
+                                             const CUtensorMap *tq1, const CUtensorMap *td1,
+                                             const CUtensorMap *tx) {
     constexpr int HALVES = MODE == kModeSwiGLU ? 2 : 1;
+    const uint64_t pw = policy_evict_first(), px = policy_evict_last();
+    // A full tile is one box of TG units for the q bytes and one for the
+    // scales (two TMA instructions: each costs tens of ns to issue); the
+    // partial last tile of a CTA's range is fetched unit by unit so that
+    // nothing outside the range is read.
+    auto issue_weights = [&](int it) {
+        const int slot = it % a.stages;
+        const int ut = u0 + (it / a.ksteps) * a.TG;
+        const int tga = min(a.TG, u1 - ut);
+        const int c0 = (it % a.ksteps) * a.CS;
+        const uint32_t st = smem_u32(smem + (size_t)slot * a.stage_bytes);
+        const uint32_t full = full0 + 8 * slot;
+        mbar_arrive_expect_tx(full, HALVES * tga * (a.q_box + a.d_box) + a.x_box);
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h) {
+            const int g0 = ut + (h ? a.up_group0 : 0);
+            const uint32_t qd = st + (h ? a.q_half : 0u), dd = st + a.d_off + (h ? a.d_half : 0u);
+            if (tga == a.TG) {
+                tma_load_3d(qd, tq, full, 0, c0, g0, pw);
+                tma_load_3d(dd, td, full, 0, c0 >> 1, g0, pw);
+            } else {
+                for (int g = 0; g < tga; ++g) {
+                    tma_load_3d(qd + g * a.q_box, tq1, full, 0, c0, g0 + g, pw);
+                    tma_load_3d(dd + g * a.d_box, td1, full, 0, c0 >> 1, g0 + g, pw);
+                }
+            }
+        }
+    };
+    auto issue_x = [&](int it) {
+        const int slot = it % a.stages;
+        const uint32_t st = smem_u32(smem + (size_t)slot * a.stage_bytes);
+        tma_load_3d(st + a.x_off, tx, full0 + 8 * slot, 0, (it % a.ksteps) * a.CS, 0, px);
+    };
+    const int pro = total < a.stages ? total : a.stages;
+    int it = 0;
+    for (; it < pro; ++it) issue_weights(it);  // weights never depend on the previous grid
+    pdl_wait();                                // activations may
+    for (int k = 0; k < pro; ++k) issue_x(k);
+    for (; it < total; ++it) {
+        const int slot = it % a.stages;
+        if (!mbar_wait(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag)) break;
+        issue_weights(it);
+        issue_x(it);
+    }
+    *issued = it;
+}
+
+// A wait gave up somewhere: make sure no copy is still landing in this CTA's
+// shared memory before it exits.
+__device__ __forceinline__ void tile_drain(uint32_t full0, const TileArgs &a, int n_issued) {
+    for (int it = n_issued > a.stages ? n_issued - a.stages : 0; it < n_issued; ++it)
+        mbar_drain(full0 + 8 * (it % a.stages), (it / a.stages) & 1);
+}
+
+// ---------------------------------------------------------------------------
+// Column-owner kernel (N <= 4)
+// ---------------------------------------------------------------------------
+// Consumer warp lw of group cg takes the 4-column quads cq = lw, lw + 8, ...
+// of every stage whose index is cg modulo the number of groups; a lane keeps
+// its column's activations in registers and runs every unit of the tile
+// against them, so each column gives TGM independent dequant + dot chains and
+// activations are read once per column.  At the end of a tile each warp
+// leaves its partial sums in a double-buffered shared area and moves on; a
+// reducer warp adds the partials of every unit in warp order and stores the
+// outputs, so no consumer ever waits on a CTA-wide barrier.
+template <int NMAX, int MODE, int CW_>
+struct ColsCfg {
+    static constexpr int CW = CW_;                           // consumer warps (8 or 16)
+    static constexpr int WPG = 8;                            // warps per consumer group
+    static constexpr int GROUPS = CW / WPG;                  // groups alternate stages
+    static constexpr int TGM = (MODE == kModeSwiGLU ? 4 : 8) / (NMAX == 4 ? 2 : 1);
+    static constexpr int H = MODE == kModeSwiGLU ? 2 : 1;
+    static constexpr int THREADS = (CW + 2) * 32;            // + producer + reducer
+    static constexpr int RED_FLOATS = 2 * CW * TGM * H * NMAX * 8;
+};
+
+// One column of every unit of the tile for lane (r, j).  GUARD = false is the
+// full-tile path: no per-unit branch, so the compiler can overlap the
+// independent per-unit chains (shared loads, dequantisation, dot products).
+template <int NMAX, int MODE, int TGM, bool GUARD>
+__device__ __forceinline__ void cols_step(const uint8_t *st, const TileArgs &a, int ks, int col,
+                                          int cols, int r, int j, int tga,
+                                          float (&acc)[TGM][MODE == kModeSwiGLU ? 2 : 1][NMAX]) {
+    constexpr int H = MODE == kModeSwiGLU ? 2 : 1;
+    if (MODE == kModeQ8Q8) {
+        // every lane takes part (the block halves meet in a shuffle); columns
+        // past K are zero-filled and add nothing
+        const int blk = min((ks * a.CS + col) >> 1, a.B - 1);
+        uint4 xv[NMAX];
+        float dx[NMAX];
+#pragma unroll
+        for (int n = 0; n < NMAX; ++n) {
+            if (n < a.N) {
+                xv[n] = *reinterpret_cast<const uint4 *>(st + a.x_off + (n * a.CS + col) * 16);
+                dx[n] = __half2float(__ushort_as_half(__ldg(a.xd + (size_t)n * a.B + blk)));
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < TGM; ++g) {
+            if (!GUARD || g < tga) {
+                const uint4 qb = *reinterpret_cast<const uint4 *>(st + g * a.q_box + col * kColBytes + r * 16);
+                const uint32_t w0 = qb.x ^ 0x80808080u, w1 = qb.y ^ 0x80808080u, w2 = qb.z ^ 0x80808080u,
+                               w3 = qb.w ^ 0x80808080u;
+                const float dw = __half2float(*reinterpret_cast<const __half *>(
+                    st + a.d_off + g * a.d_slot + (col >> 1) * 16 + r * 2));
+#pragma unroll
+                for (int n = 0; n < NMAX; ++n) {
+                    if (n < a.N) {
+                        int dot = dp4a_s8(w0, xv[n].x, 0);
+                        dot = dp4a_s8(w1, xv[n].y, dot);
+                        dot = dp4a_s8(w2, xv[n].z, dot);
+                        dot = dp4a_s8(w3, xv[n].w, dot);
+                        dot += __shfl_xor_sync(0xffffffffu, dot, 8);
+                        if ((j & 1) == 0) acc[g][0][n] = fmaf((float)dot, dw * dx[n], acc[g][0][n]);
+                    }
+                }
+            }
+        }
+    } else if (col < cols) {
+        ulonglong2 xr[NMAX][4];
+#pragma unroll
+        for (int n = 0; n < NMAX; ++n) {
+            if (n < a.N) {
+                const ulonglong2 *xv = reinterpret_cast<const ulonglong2 *>(st + a.x_off + (n * a.CS + col) * 64);
+                xr[n][0] = xv[0];
+                xr[n][1] = xv[1];
+                xr[n][2] = xv[2];
+                xr[n][3] = xv[3];
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < TGM; ++g) {
+            if (!GUARD || g < tga) {
+#pragma unroll
+                for (int h = 0; h < H; ++h) {
+                    ColPiece pc;
+                    load_piece(st, a, h ? a.q_half : 0u, h ? a.d_half : 0u, g, col, r, pc);
+#pragma unroll
+                    for (int n = 0; n < NMAX; ++n)
+                        if (n < a.N)
+                            acc[g][h][n] = fmaf(dot16_x2(pc.w, xr[n][0], xr[n][1], xr[n][2], xr[n][3]), pc.d,
+                                                acc[g][h][n]);
+                }
+            }
+        }
+    }
+}
+
+template <int NMAX, int MODE, int CW_>
+__global__ void __launch_bounds__(ColsCfg<NMAX, MODE, CW_>::THREADS, 1)
+    cols_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap td,
+                const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap td1,
+                const __grid_constant__ CUtensorMap tx, const TileArgs a) {
+    using Cfg = ColsCfg<NMAX, MODE, CW_>;
+    constexpr int TGM = Cfg::TGM, H = Cfg::H, CW = Cfg::CW, WPG = Cfg::WPG;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)a.stages * a.stage_bytes);
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + a.stages);
-    float *red = reinterpret_cast<float *>(bars + 2 * a.stages);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(red + tile_red_floats(NMAX, SETS));
+    const uint32_t redfull0 = smem_u32(bars + 2 * a.stages), redfree0 = redfull0 + 16;
+    float *red = reinterpret_cast<float *>(bars + 2 * a.stages + 4);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(red + Cfg::RED_FLOATS);
     volatile int *issued = abort_flag + 1;
 
+    // units * grid < 2^31 is checked on the host, so 32-bit math is exact here
+    const int u0 = (int)(((unsigned)a.units * blockIdx.x) / gridDim.x);
+    const int u1 = (int)(((unsigned)a.units * (blockIdx.x + 1)) / gridDim.x);
+    const int n_tiles = (u1 - u0 + a.TG - 1) / a.TG;
+    const int total = n_tiles * a.ksteps;
+    const int used_stages = total < a.stages ? total : a.stages;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < a.stages; ++s) {
+        for (int s = 0; s < used_stages; ++s) {
             mbar_init(full0 + 8 * s, 1);
-            mbar_init(empty0 + 8 * s, kConsumerWarps);
+            mbar_init(empty0 + 8 * s, WPG);
+        }
+        for (int p = 0; p < 2; ++p) {
+            mbar_init(redfull0 + 8 * p, CW);
+            mbar_init(redfree0 + 8 * p, 1);
         }
         *abort_flag = 0;
         *issued = 0;
@@ -201,109 +372,66 @@ __global__ void __launch_bounds__(kTileThreads, 1)
     // nothing this kernel writes before its own griddepcontrol.wait.
     pdl_launch_dependents();
 
-    const int u0 = (int)(((int64_t)a.units * blockIdx.x) / gridDim.x);
-    const int u1 = (int)(((int64_t)a.units * (blockIdx.x + 1)) / gridDim.x);
-    const int n_tiles = (u1 - u0 + a.TG - 1) / a.TG;
-    const int total = n_tiles * a.ksteps;
-
-    if (warp == kConsumerWarps) {
-        // ------------------------------ producer ------------------------------
-        if (lane == 0) {
-            prefetch_tensormap(&tq);
-            prefetch_tensormap(&td);
-            prefetch_tensormap(&tx);
-            const uint64_t pw = policy_evict_first(), px = policy_evict_last();
-            auto issue_weights = [&](int it) {
-                const int slot = it % a.stages;
-                const int ut = u0 + (it / a.ksteps) * a.TG;
-                const int tga = min(a.TG, u1 - ut);
-                const int c0 = (it % a.ksteps) * a.CS;
-                const uint32_t st = smem_u32(smem + (size_t)slot * a.stage_bytes);
-                const uint32_t full = full0 + 8 * slot;
-                mbar_arrive_expect_tx(full, HALVES * tga * (a.q_box + a.d_box) + a.x_box);
-                for (int g = 0; g < tga; ++g) {
-                    tma_load_3d(st + g * a.q_box, &tq, full, 0, c0, ut + g, pw);
-                    tma_load_3d(st + a.d_off + g * a.d_slot, &td, full, 0, c0 >> 1, ut + g, pw);
-                    if (MODE == kModeSwiGLU) {
-                        tma_load_3d(st + a.q_half + g * a.q_box, &tq, full, 0, c0,
-                                    ut + g + a.up_group0, pw);
-                        tma_load_3d(st + a.d_off + a.d_half + g * a.d_slot, &td, full, 0, c0 >> 1,
-                                    ut + g + a.up_group0, pw);
-                    }
+    if (warp == CW) {
+        if (lane == 0)
+            tile_produce<MODE>(smem, full0, empty0, abort_flag, issued, a, u0, u1, total, &tq, &td,
+                               &tq1, &td1, &tx);
+    } else if (warp == CW + 1) {
+        // ------------------------------ reducer -------------------------------
+        pdl_wait();  // the outputs may still be read by the previous grid
+        for (int tl = 0; tl < n_tiles; ++tl) {
+            const int p = tl & 1;
+            const bool ok = mbar_wait(redfull0 + 8 * p, (tl >> 1) & 1, abort_flag);
+            const int ut = u0 + tl * a.TG;
+            const int tga = min(a.TG, u1 - ut);
+            if (ok) {
+                for (int o = lane; o < tga * 8; o += 32) {
+                    const int g = o >> 3, rr = o & 7;
+                    float v[H][NMAX];
+#pragma unroll
+                    for (int h = 0; h < H; ++h)
+#pragma unroll
+                        for (int n = 0; n < NMAX; ++n) {
+                            float sum = 0.f;
+#pragma unroll
+                            for (int w = 0; w < CW; ++w)
+                                sum += red[(((((p * CW + w) * TGM + g) * H + h) * NMAX + n) << 3) + rr];
+                            v[h][n] = sum;
+                        }
+                    store_unit<NMAX, MODE>(a, ut + g, rr, v[0], v[H - 1]);
                 }
-            };
-            auto issue_x = [&](int it) {
-                const int slot = it % a.stages;
-                const uint32_t st = smem_u32(smem + (size_t)slot * a.stage_bytes);
-                tma_load_3d(st + a.x_off, &tx, full0 + 8 * slot, 0, (it % a.ksteps) * a.CS, 0, px);
-            };
-            const int pro = total < a.stages ? total : a.stages;
-            int it = 0;
-            for (; it < pro; ++it) issue_weights(it);  // weights never depend on the previous grid
-            pdl_wait();                                // activations may
-            for (int k = 0; k < pro; ++k) issue_x(k);
-            for (; it < total; ++it) {
-                const int slot = it % a.stages;
-                if (!mbar_wait(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag)) break;
-                issue_weights(it);
-                issue_x(it);
             }
-            *issued = it;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(redfree0 + 8 * p);
         }
     } else {
         // ------------------------------ consumers -----------------------------
-        const int cw = warp, r = lane & 7, j = lane >> 3;
-        pdl_wait();  // outputs may still be read by the previous grid
+        const int cw = warp, cg = cw / WPG, lw = cw % WPG, r = lane & 7, j = lane >> 3;
+        if (MODE == kModeQ8Q8) pdl_wait();  // activation scales are read straight from memory
         int it = 0;
         for (int tl = 0; tl < n_tiles; ++tl) {
             const int ut = u0 + tl * a.TG;
             const int tga = min(a.TG, u1 - ut);
-            const bool whole = tga >= 8;  // each warp owns whole units
-            // split mode: this warp's contiguous range of (unit, quad) pairs
-            const int P = tga * a.NQ;
-            const int p_lo = (P * cw) / kConsumerWarps, p_hi = (P * (cw + 1)) / kConsumerWarps;
-            const int gs0 = p_lo / a.NQ;
-            const int gs1 = p_hi > p_lo ? (p_hi - 1) / a.NQ : gs0;
-            float acc[SETS][NMAX];
+            float acc[TGM][H][NMAX];
 #pragma unroll
-            for (int h = 0; h < SETS; ++h)
+            for (int g = 0; g < TGM; ++g)
 #pragma unroll
-                for (int n = 0; n < NMAX; ++n) acc[h][n] = 0.f;
+                for (int h = 0; h < H; ++h)
+#pragma unroll
+                    for (int n = 0; n < NMAX; ++n) acc[g][h][n] = 0.f;
             for (int ks = 0; ks < a.ksteps; ++ks, ++it) {
+                if (it % Cfg::GROUPS != cg) continue;
                 const int slot = it % a.stages;
                 if (mbar_wait(full0 + 8 * slot, (it / a.stages) & 1, abort_flag)) {
                     const uint8_t *st = smem + (size_t)slot * a.stage_bytes;
                     const int cols = min(a.CS, a.C - ks * a.CS);
                     const int nq = (cols + 3) >> 2;
-                    if (whole) {
-                        const int gB = cw + 8 < tga ? cw + 8 : -1;
-                        for (int cq = 0; cq < nq; ++cq) {
-                            const int col = 4 * cq + j;
-                            if (MODE == kModeF32 && gB >= 0) {
-                                if (col < cols) {
-                                    ColPiece p0, p1;
-                                    load_piece(st, a, 0, 0, cw, col, r, p0);
-                                    load_piece(st, a, 0, 0, gB, col, r, p1);
-                                    fp32_column<NMAX>(st, a, col, p0, &p1, acc[0], acc[1]);
-                                }
-                            } else if (MODE == kModeQ8Q8 || col < cols) {
-                                unit_column<NMAX, MODE>(st, a, ks, col, r, j, cw, 0, acc);
-                                if (gB >= 0) unit_column<NMAX, MODE>(st, a, ks, col, r, j, gB, 1, acc);
-                            }
-                        }
-                    } else {
-                        const int qs0 = ks * (a.CS >> 2);
-                        for (int s = 0; s < 2; ++s) {
-                            const int g = s == 0 ? gs0 : gs1;
-                            if (s == 1 && gs1 == gs0) break;
-                            const int lo = max(max(p_lo - g * a.NQ, 0), qs0);
-                            const int hi = min(min(p_hi - g * a.NQ, a.NQ), qs0 + nq);
-                            for (int qk = lo; qk < hi; ++qk) {
-                                const int col = 4 * (qk - qs0) + j;
-                                if (MODE == kModeQ8Q8 || col < cols)
-                                    unit_column<NMAX, MODE>(st, a, ks, col, r, j, g, s, acc);
-                            }
-                        }
+                    for (int cq = lw; cq < nq; cq += WPG) {
+                        const int col = 4 * cq + j;
+                        if (tga == TGM)
+                            cols_step<NMAX, MODE, TGM, false>(st, a, ks, col, cols, r, j, tga, acc);
+                        else
+                            cols_step<NMAX, MODE, TGM, true>(st, a, ks, col, cols, r, j, tga, acc);
                     }
                 }
                 __syncwarp();
@@ -311,61 +439,188 @@ __global__ void __launch_bounds__(kTileThreads, 1)
             }
             // lanes r, r+8, r+16, r+24 hold partial sums of the same row
 #pragma unroll
-            for (int h = 0; h < SETS; ++h)
+            for (int g = 0; g < TGM; ++g)
 #pragma unroll
-                for (int n = 0; n < NMAX; ++n) {
-                    acc[h][n] += __shfl_xor_sync(0xffffffffu, acc[h][n], 8);
-                    acc[h][n] += __shfl_xor_sync(0xffffffffu, acc[h][n], 16);
-                }
-            if (whole) {
-                if (j == 0) {
-                    if (MODE == kModeSwiGLU) {
-                        store_unit<NMAX, MODE>(a, ut + cw, r, acc[0], acc[1]);
-                    } else {
-                        store_unit<NMAX, MODE>(a, ut + cw, r, acc[0], acc[0]);
-                        if (cw + 8 < tga) store_unit<NMAX, MODE>(a, ut + cw + 8, r, acc[1], acc[1]);
+                for (int h = 0; h < H; ++h)
+#pragma unroll
+                    for (int n = 0; n < NMAX; ++n) {
+                        acc[g][h][n] += __shfl_xor_sync(0xffffffffu, acc[g][h][n], 8);
+                        acc[g][h][n] += __shfl_xor_sync(0xffffffffu, acc[g][h][n], 16);
                     }
-                }
-            } else {
-                if (j == 0) {
+            const int p = tl & 1;
+            if (tl >= 2) mbar_wait(redfree0 + 8 * p, ((tl >> 1) - 1) & 1, abort_flag);
+            if (j == 0) {
 #pragma unroll
-                    for (int h = 0; h < SETS; ++h)
+                for (int g = 0; g < TGM; ++g)
 #pragma unroll
-                        for (int n = 0; n < NMAX; ++n) red[((cw * SETS + h) * NMAX + n) * 8 + r] = acc[h][n];
-                }
-                named_barrier(1, kConsumerWarps * 32);
-                if (cw < tga && j == 0) {
-                    // unit cw: add the partials of every warp whose range touches it, in warp order
-                    constexpr int PER = SETS / 2;  // accumulator sets per unit slot
-                    float v[PER][NMAX];
+                    for (int h = 0; h < H; ++h)
 #pragma unroll
-                    for (int h = 0; h < PER; ++h)
-#pragma unroll
-                        for (int n = 0; n < NMAX; ++n) v[h][n] = 0.f;
-                    for (int w = 0; w < kConsumerWarps; ++w) {
-                        const int wl = (P * w) / kConsumerWarps, wh = (P * (w + 1)) / kConsumerWarps;
-                        if (wh <= wl || wl >= (cw + 1) * a.NQ || wh <= cw * a.NQ) continue;
-                        const int slot = (wl / a.NQ == cw) ? 0 : 1;
-#pragma unroll
-                        for (int h = 0; h < PER; ++h)
-#pragma unroll
-                            for (int n = 0; n < NMAX; ++n)
-                                v[h][n] += red[((w * SETS + slot * PER + h) * NMAX + n) * 8 + r];
-                    }
-                    store_unit<NMAX, MODE>(a, ut + cw, r, v[0], v[PER - 1]);
-                }
-                named_barrier(1, kConsumerWarps * 32);
+                        for (int n = 0; n < NMAX; ++n)
+                            red[(((((p * CW + cw) * TGM + g) * H + h) * NMAX + n) << 3) + r] = acc[g][h][n];
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(redfull0 + 8 * p);
         }
     }
     __syncthreads();
-    if (threadIdx.x == 0 && *abort_flag) {
-        // A wait gave up: make sure no copy is still landing in this CTA's
-        // shared memory before it exits.
-        const int n_issued = *issued;
-        for (int it = n_issued > a.stages ? n_issued - a.stages : 0; it < n_issued; ++it)
-            mbar_drain(full0 + 8 * (it % a.stages), (it / a.stages) & 1);
+    if (threadIdx.x == 0 && *abort_flag) tile_drain(full0, a, *issued);
+}
+
+// ---------------------------------------------------------------------------
+// Group-owner kernel (N >= 5)
+// ---------------------------------------------------------------------------
+// Group owners (N >= 5): a tile of >= 8 units gives each warp one or two whole
+// units (no cross-warp traffic); a smaller tile splits its (unit, quad) pairs
+// evenly over the warps and adds their partial sums in warp order.
+template <int NMAX, int MODE>
+__device__ __forceinline__ void consume_groups(uint8_t *smem, uint32_t full0, uint32_t empty0,
+                                               float *red, volatile int *abort_flag,
+                                               const TileArgs &a, int u0, int u1, int n_tiles) {
+    constexpr int SETS = tile_acc_sets<MODE>();
+    const int cw = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane & 7, j = lane >> 3;
+    pdl_wait();  // outputs may still be read by the previous grid
+    int it = 0;
+    for (int tl = 0; tl < n_tiles; ++tl) {
+        const int ut = u0 + tl * a.TG;
+        const int tga = min(a.TG, u1 - ut);
+        const bool whole = tga >= 8;
+        const int P = tga * a.NQ;
+        const int p_lo = (P * cw) / kConsumerWarps, p_hi = (P * (cw + 1)) / kConsumerWarps;
+        const int gs0 = p_lo / a.NQ;
+        const int gs1 = p_hi > p_lo ? (p_hi - 1) / a.NQ : gs0;
+        float acc[SETS][NMAX];
+#pragma unroll
+        for (int h = 0; h < SETS; ++h)
+#pragma unroll
+            for (int n = 0; n < NMAX; ++n) acc[h][n] = 0.f;
+        for (int ks = 0; ks < a.ksteps; ++ks, ++it) {
+            const int slot = it % a.stages;
+            if (mbar_wait(full0 + 8 * slot, (it / a.stages) & 1, abort_flag)) {
+                const uint8_t *st = smem + (size_t)slot * a.stage_bytes;
+                const int cols = min(a.CS, a.C - ks * a.CS);
+                const int nq = (cols + 3) >> 2;
+                if (whole) {
+                    const int gB = cw + 8 < tga ? cw + 8 : -1;
+                    for (int cq = 0; cq < nq; ++cq) {
+                        const int col = 4 * cq + j;
+                        if (MODE == kModeF32 && gB >= 0) {
+                            if (col < cols) {
+                                ColPiece p0, p1;
+                                load_piece(st, a, 0, 0, cw, col, r, p0);
+                                load_piece(st, a, 0, 0, gB, col, r, p1);
+                                fp32_column<NMAX>(st, a, col, p0, &p1, acc[0], acc[1]);
+                            }
+                        } else if (MODE == kModeQ8Q8 || col < cols) {
+                            unit_column<NMAX, MODE>(st, a, ks, col, r, j, cw, 0, acc);
+                            if (gB >= 0) unit_column<NMAX, MODE>(st, a, ks, col, r, j, gB, 1, acc);
+                        }
+                    }
+                } else {
+                    const int qs0 = ks * (a.CS >> 2);
+                    for (int s = 0; s < 2; ++s) {
+                        const int g = s == 0 ? gs0 : gs1;
+                        if (s == 1 && gs1 == gs0) break;
+                        const int lo = max(max(p_lo - g * a.NQ, 0), qs0);
+                        const int hi = min(min(p_hi - g * a.NQ, a.NQ), qs0 + nq);
+                        for (int qk = lo; qk < hi; ++qk) {
+                            const int col = 4 * (qk - qs0) + j;
+                            if (MODE == kModeQ8Q8 || col < cols)
+                                unit_column<NMAX, MODE>(st, a, ks, col, r, j, g, s, acc);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty0 + 8 * slot);
+        }
+#pragma unroll
+        for (int h = 0; h < SETS; ++h)
+#pragma unroll
+            for (int n = 0; n < NMAX; ++n) {
+                acc[h][n] += __shfl_xor_sync(0xffffffffu, acc[h][n], 8);
+                acc[h][n] += __shfl_xor_sync(0xffffffffu, acc[h][n], 16);
+            }
+        if (whole) {
+            if (j == 0) {
+                if (MODE == kModeSwiGLU) {
+                    store_unit<NMAX, MODE>(a, ut + cw, r, acc[0], acc[1]);
+                } else {
+                    store_unit<NMAX, MODE>(a, ut + cw, r, acc[0], acc[0]);
+                    if (cw + 8 < tga) store_unit<NMAX, MODE>(a, ut + cw + 8, r, acc[1], acc[1]);
+                }
+            }
+        } else {
+            if (j == 0) {
+#pragma unroll
+                for (int h = 0; h < SETS; ++h)
+#pragma unroll
+                    for (int n = 0; n < NMAX; ++n) red[((cw * SETS + h) * NMAX + n) * 8 + r] = acc[h][n];
+            }
+            named_barrier(1, kConsumerWarps * 32);
+            if (cw < tga && j == 0) {
+                constexpr int PER = SETS / 2;
+                float v[PER][NMAX];
+#pragma unroll
+                for (int h = 0; h < PER; ++h)
+#pragma unroll
+                    for (int n = 0; n < NMAX; ++n) v[h][n] = 0.f;
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const int wl = (P * w) / kConsumerWarps, wh = (P * (w + 1)) / kConsumerWarps;
+                    if (wh <= wl || wl >= (cw + 1) * a.NQ || wh <= cw * a.NQ) continue;
+                    const int slot = (wl / a.NQ == cw) ? 0 : 1;
+#pragma unroll
+                    for (int h = 0; h < PER; ++h)
+#pragma unroll
+                        for (int n = 0; n < NMAX; ++n)
+                            v[h][n] += red[((w * SETS + slot * PER + h) * NMAX + n) * 8 + r];
+                }
+                store_unit<NMAX, MODE>(a, ut + cw, r, v[0], v[PER - 1]);
+            }
+            named_barrier(1, kConsumerWarps * 32);
+        }
     }
+}
+
+template <int NMAX, int MODE>
+__global__ void __launch_bounds__(kTileThreads, 1)
+    tile_gemm_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap td,
+                     const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap td1,
+                     const __grid_constant__ CUtensorMap tx, const TileArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)a.stages * a.stage_bytes);
+    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + a.stages);
+    float *red = reinterpret_cast<float *>(bars + 2 * a.stages);
+    volatile int *abort_flag =
+        reinterpret_cast<volatile int *>(red + tile_red_floats(NMAX, tile_acc_sets<MODE>()));
+    volatile int *issued = abort_flag + 1;
+
+    const int u0 = (int)(((unsigned)a.units * blockIdx.x) / gridDim.x);
+    const int u1 = (int)(((unsigned)a.units * (blockIdx.x + 1)) / gridDim.x);
+    const int n_tiles = (u1 - u0 + a.TG - 1) / a.TG;
+    const int total = n_tiles * a.ksteps;
+    const int used_stages = total < a.stages ? total : a.stages;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < used_stages; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, kConsumerWarps);
+        }
+        *abort_flag = 0;
+        *issued = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+
+    if (warp == kConsumerWarps) {
+        if (lane == 0)
+            tile_produce<MODE>(smem, full0, empty0, abort_flag, issued, a, u0, u1, total, &tq, &td,
+                               &tq1, &td1, &tx);
+    } else {
+        consume_groups<NMAX, MODE>(smem, full0, empty0, red, abort_flag, a, u0, u1, n_tiles);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag) tile_drain(full0, a, *issued);
 }
 
 }  // namespace q8
