@@ -10,6 +10,7 @@
 #include "q8q8.cuh"
 #include "route.cuh"
 #include "tile_gemm.cuh"
+#include "moe.cuh"
 
 namespace q8 {
 
@@ -210,6 +211,88 @@ static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, floa
                       tx, a);
 }
 
+// ---------------------------------------------------------------------------
+// grouped MoE (S6)
+// ---------------------------------------------------------------------------
+using MoeKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+                           CUtensorMap, MoeArgs);
+
+template <int STAGE, int NMAX>
+static MoeKernel moe_kernel_ptr() {
+    constexpr int TGM = STAGE == 1 ? (32 / NMAX < 1 ? 1 : 32 / NMAX > 8 ? 8 : 32 / NMAX)
+                                   : (64 / NMAX > 8 ? 8 : 64 / NMAX);
+    return &moe_kernel<STAGE, NMAX, TGM>;
+}
+
+static int moe_tgm(int stage, int nmax) {
+    const int v = (stage == 1 ? 32 : 64) / nmax;
+    return v < 1 ? 1 : v > 8 ? 8 : v;
+}
+
+static MoeKernel moe_kernel_for(int stage, int nmax) {
+    switch (nmax) {
+        case 1: return stage == 1 ? moe_kernel_ptr<1, 1>() : moe_kernel_ptr<2, 1>();
+        case 2: return stage == 1 ? moe_kernel_ptr<1, 2>() : moe_kernel_ptr<2, 2>();
+        case 4: return stage == 1 ? moe_kernel_ptr<1, 4>() : moe_kernel_ptr<2, 4>();
+        case 8: return stage == 1 ? moe_kernel_ptr<1, 8>() : moe_kernel_ptr<2, 8>();
+        default: return stage == 1 ? moe_kernel_ptr<1, 16>() : moe_kernel_ptr<2, 16>();
+    }
+}
+
+static cudaError_t setup_moe_kernels(int max_smem) {
+    const int nm[5] = {1, 2, 4, 8, 16};
+    for (int i = 0; i < 5; ++i)
+        for (int stage = 1; stage <= 2; ++stage) {
+            const void *k = reinterpret_cast<const void *>(moe_kernel_for(stage, nm[i]));
+            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+            if (e != cudaSuccess) return e;
+            e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared);
+            if (e != cudaSuccess) return e;
+        }
+    return cudaSuccess;
+}
+static RegisterSetup g_reg_moe(setup_moe_kernels);
+
+struct MoePlan {
+    MoeArgs a;
+    int grid;
+    size_t smem;
+};
+
+// Stage shape for a MoE launch: TG units of `halves` weight boxes of CS
+// columns (~32 KB) plus the activation box of T rows (<= 16 KB).
+static MoePlan plan_moe(int stage, int64_t T, int64_t c_min, int nmax, int64_t units_bound, int sms) {
+    MoePlan p;
+    MoeArgs &a = p.a;
+    a = MoeArgs{};
+    const int halves = stage == 1 ? 2 : 1;
+    const int tg = moe_tgm(stage, nmax);
+    int64_t cs = (32 * 1024) / ((int64_t)tg * halves * 136) / 16 * 16;
+    const int64_t cs_x = (16 * 1024) / (T * 64) / 16 * 16;
+    cs = std::min<int64_t>(cs, cs_x);
+    cs = std::min<int64_t>(cs, round_up(c_min, 16));
+    if (cs < 16) cs = 16;
+    a.TG = tg;
+    a.CS = (int)cs;
+    a.q_box = (uint32_t)(cs * kColBytes);
+    a.d_box = (uint32_t)(cs * 8);
+    a.x_box = (uint32_t)(T * cs * 64);
+    a.q_half = (uint32_t)tg * a.q_box;
+    a.d_off = halves * a.q_half;
+    a.d_half = (uint32_t)tg * a.d_box;
+    a.x_off = a.d_off + halves * a.d_half;
+    a.stage_bytes = (uint32_t)round_up(a.x_off + a.x_box, 128);
+    const size_t fixed = sizeof(MoeTable) + (size_t)kMoeWarps * tg * halves * nmax * 8 * 4 + 16;
+    int64_t stages = (int64_t)(104 * 1024 - fixed) / a.stage_bytes;
+    a.stages = (int)(stages < 2 ? 2 : stages > 6 ? 6 : stages);
+    p.grid = (int)std::min<int64_t>(sms, units_bound);
+    p.smem = (size_t)a.stages * a.stage_bytes + 16 * a.stages + fixed;
+    return p;
+}
+
+static size_t moe_hbuf_bytes(int64_t T, int64_t k, int64_t I) { return (size_t)round_up(T * k * I * 4, 256); }
+
 }  // namespace q8
 
 using namespace q8;
@@ -361,8 +444,8 @@ q8_status q8_moe_route(const float *logits, int64_t T, int64_t E, int64_t top_k,
 
 size_t q8_moe_workspace_bytes(int64_t T, int64_t E, int64_t top_k, int64_t H, int64_t I,
                               int64_t I_shared) {
-    (void)T; (void)E; (void)top_k; (void)H; (void)I; (void)I_shared;
-    return 0;
+    if (T <= 0 || E <= 0 || top_k <= 0 || H <= 0 || I <= 0 || I_shared < 0) return 0;
+    return moe_hbuf_bytes(T, top_k, I) + (size_t)round_up(T * I_shared * 4, 256);
 }
 
 q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
@@ -370,10 +453,100 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
                       const int32_t *idx, const float *w, const float *x, float *y, int64_t T,
                       int64_t E, int64_t top_k, int64_t H, int64_t I, int64_t I_shared,
                       void *workspace, size_t workspace_bytes, q8_stream_t stream) {
-    (void)gate_up_experts; (void)down_experts; (void)shared_gate_up; (void)shared_down;
-    (void)idx; (void)w; (void)x; (void)y; (void)T; (void)E; (void)top_k; (void)H; (void)I;
-    (void)I_shared; (void)workspace; (void)workspace_bytes; (void)stream;
-    return Q8_ERR_UNSUPPORTED;
+    if (T <= 0 || E <= 0 || top_k <= 0 || top_k > E || H <= 0 || I <= 0 || I_shared < 0)
+        return Q8_ERR_SHAPE;
+    if (H % 32 || I % 32 || I_shared % 32) return Q8_ERR_SHAPE;
+    if (T > kMoeMaxT || top_k > kMoeMaxK || E > kMoeMaxE || H > 65536 || I > 65536 ||
+        I_shared > 65536)
+        return Q8_ERR_UNSUPPORTED;
+    const bool has_shared = shared_gate_up != nullptr || shared_down != nullptr;
+    if (has_shared != (I_shared > 0) || (has_shared && (!shared_gate_up || !shared_down)))
+        return Q8_ERR_INVALID;
+    Q8_CHECK(check_device_ptr(gate_up_experts));
+    Q8_CHECK(check_device_ptr(down_experts));
+    if (has_shared) {
+        Q8_CHECK(check_device_ptr(shared_gate_up));
+        Q8_CHECK(check_device_ptr(shared_down));
+    }
+    Q8_CHECK(check_device_ptr(idx, false));
+    Q8_CHECK(check_device_ptr(w, false));
+    if ((reinterpret_cast<uintptr_t>(idx) | reinterpret_cast<uintptr_t>(w)) & 3u) return Q8_ERR_ALIGN;
+    Q8_CHECK(check_device_ptr(x));
+    Q8_CHECK(check_device_ptr(y));
+    Q8_CHECK(check_device_ptr(workspace));
+    if (workspace_bytes < q8_moe_workspace_bytes(T, E, top_k, H, I, I_shared)) return Q8_ERR_SHAPE;
+    const DeviceInfo *dev = nullptr;
+    Q8_CHECK(device_info(&dev));
+    cudaStream_t s = (cudaStream_t)stream;
+    float *hbuf = static_cast<float *>(workspace);
+    float *hsh = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + moe_hbuf_bytes(T, top_k, I));
+    const int nb = nmax_for(T);
+    const int64_t Ish = has_shared ? I_shared : 0;
+
+    // ---- launch 1: gate_up + SwiGLU over selected experts and the shared one
+    {
+        const int64_t units_bound = std::min<int64_t>(T * top_k, E) * (I / 8) + Ish / 8;
+        MoePlan p = plan_moe(1, T, H / 16, nb, units_bound, dev->sms);
+        MoeArgs &a = p.a;
+        a.T = (int)T; a.E = (int)E; a.k = (int)top_k; a.H = (int)H; a.I = (int)I; a.Is = (int)Ish;
+        a.idx = idx; a.w = w; a.hbuf = hbuf; a.hsh = hsh; a.y = y;
+        a.units_out = (int)(H / 8);
+        if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
+        const uint64_t gs = (uint64_t)kGroupBytesPerBlock * (H / 32);
+        CUtensorMap tq_r, td_r, tq_s, td_s, tx;
+        Q8_CHECK(make_map_3d(&tq_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, gate_up_experts, kColBytes, H / 16,
+                             E * (2 * I / 8), kColBytes, gs, kColBytes, a.CS, 1, true));
+        Q8_CHECK(make_map_3d(&td_r, CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                             static_cast<const uint8_t *>(gate_up_experts) + 256 * (H / 32), 8, H / 32,
+                             E * (2 * I / 8), 16, gs, 8, a.CS / 2, 1, true));
+        const void *sgu = has_shared ? shared_gate_up : gate_up_experts;
+        const int64_t sg = has_shared ? 2 * Ish / 8 : E * (2 * I / 8);
+        Q8_CHECK(make_map_3d(&tq_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, sgu, kColBytes, H / 16, sg, kColBytes, gs,
+                             kColBytes, a.CS, 1, true));
+        Q8_CHECK(make_map_3d(&td_s, CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                             static_cast<const uint8_t *>(sgu) + 256 * (H / 32), 8, H / 32, sg, 16, gs, 8,
+                             a.CS / 2, 1, true));
+        Q8_CHECK(make_map_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, H / 16, T, 64, (uint64_t)H * 4, 16,
+                             a.CS, (uint32_t)T, false));
+        Q8_CHECK(launch_pdl(moe_kernel_for(1, nb), dim3(p.grid), dim3(kMoeThreads), p.smem, s,
+                            "q8_moe_gemv gate_up launch", tq_r, td_r, tq_s, td_s, tx, tx, a));
+    }
+    // ---- launch 2: down projections, summed per output row group
+    {
+        const int64_t c_min = has_shared ? std::min<int64_t>(I, Ish) / 16 : I / 16;
+        MoePlan p = plan_moe(2, T, c_min, nb, H / 8, dev->sms);
+        MoeArgs &a = p.a;
+        a.T = (int)T; a.E = (int)E; a.k = (int)top_k; a.H = (int)H; a.I = (int)I; a.Is = (int)Ish;
+        a.idx = idx; a.w = w; a.hbuf = hbuf; a.hsh = hsh; a.y = y;
+        a.units_out = (int)(H / 8);
+        if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
+        const uint64_t gs_r = (uint64_t)kGroupBytesPerBlock * (I / 32);
+        CUtensorMap tq_r, td_r, tq_s, td_s, tx_r, tx_s;
+        Q8_CHECK(make_map_3d(&tq_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, down_experts, kColBytes, I / 16,
+                             E * (H / 8), kColBytes, gs_r, kColBytes, a.CS, 1, true));
+        Q8_CHECK(make_map_3d(&td_r, CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                             static_cast<const uint8_t *>(down_experts) + 256 * (I / 32), 8, I / 32,
+                             E * (H / 8), 16, gs_r, 8, a.CS / 2, 1, true));
+        Q8_CHECK(make_map_3d(&tx_r, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, hbuf, 16, I / 16, T * top_k, 64,
+                             (uint64_t)I * 4, 16, a.CS, (uint32_t)T, false));
+        if (has_shared) {
+            const uint64_t gs_s = (uint64_t)kGroupBytesPerBlock * (Ish / 32);
+            Q8_CHECK(make_map_3d(&tq_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, shared_down, kColBytes, Ish / 16, H / 8,
+                                 kColBytes, gs_s, kColBytes, a.CS, 1, true));
+            Q8_CHECK(make_map_3d(&td_s, CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                                 static_cast<const uint8_t *>(shared_down) + 256 * (Ish / 32), 8, Ish / 32,
+                                 H / 8, 16, gs_s, 8, a.CS / 2, 1, true));
+            Q8_CHECK(make_map_3d(&tx_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, hsh, 16, Ish / 16, T, 64,
+                                 (uint64_t)Ish * 4, 16, a.CS, (uint32_t)T, false));
+        } else {
+            tq_s = tq_r;
+            td_s = td_r;
+            tx_s = tx_r;
+        }
+        Q8_CHECK(launch_pdl(moe_kernel_for(2, nb), dim3(p.grid), dim3(kMoeThreads), p.smem, s,
+                            "q8_moe_gemv down launch", tq_r, td_r, tq_s, td_s, tx_r, tx_s, a));
+    }
+    return Q8_OK;
 }
 
 }  // extern "C"
