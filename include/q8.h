@@ -169,8 +169,9 @@ size_t q8_moe_workspace_bytes(int64_t T, int64_t E, int64_t top_k, int64_t H, in
  * weighting and shared expert follow the router + top-k expert +
  * shared-expert FFN block of "Add Qwen1.5-MoE Q8_0 ... - #144" (PR summary);
  * folding the per-slot launches into one grid follows the routed-expert
- * launch fusion in that PR's conversation.  The sum over slots runs in slot
- * order for every output, so results are bit-identical from run to run.
+ * launch fusion in that PR's conversation.  Every output is summed in a fixed
+ * order (routed experts by ascending expert id, then the shared expert), so
+ * results are bit-identical from run to run.
  *   gate_up_experts: E consecutive packed matrices [2I][H], each
  *       q8_packed_bytes(2I, H) bytes (gate rows first, as q8_gate_up_swiglu).
  *   down_experts:    E consecutive packed matrices [H][I], each
@@ -188,6 +189,31 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
                       const int32_t *idx, const float *w, const float *x, float *y, int64_t T,
                       int64_t E, int64_t top_k, int64_t H, int64_t I, int64_t I_shared,
                       void *workspace, size_t workspace_bytes, q8_stream_t stream);
+
+/* Same product as q8_moe_gemv, without a workspace argument.  The pages have
+ * no counterpart: this variant exists for callers that cannot allocate device
+ * memory when they call -- for example a plug-in that is handed finished
+ * device buffers by a host framework owning the memory pool, code that runs
+ * while a stream is being captured into a CUDA graph (allocation calls are
+ * not permitted there), or a decode loop that must not risk an allocation's
+ * implicit synchronisation.
+ * Scratch comes from a fixed 4 MiB array in the library's device memory, held
+ * by every GPU that loads the library until the process exits.  Sizes whose
+ * q8_moe_workspace_bytes() exceeds 4 MiB are rejected with
+ * Q8_ERR_UNSUPPORTED (q8_last_cuda_error() gives the byte counts).  Nothing is
+ * allocated or freed.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents; the
+ * kernels write every scratch element before reading it, so nothing needs
+ * clearing between calls.  Calls that may run at the same time on the GPU
+ * (different streams without an ordering between them) race on the array and
+ * must not be issued. */
+q8_status q8_moe_gemv_noalloc(const void *gate_up_experts, const void *down_experts,
+                              const void *shared_gate_up, const void *shared_down,
+                              const int32_t *idx, const float *w, const float *x, float *y,
+                              int64_t T, int64_t E, int64_t top_k, int64_t H, int64_t I,
+                              int64_t I_shared, q8_stream_t stream);
 
 /* ---------------------------------------------------------------------- */
 /* S7  Activation quantisation to Q8_0                                     */

@@ -20,6 +20,7 @@ __all__ = [
     "Q8Error", "lib_path", "q8_status_string", "q8_last_cuda_error", "q8_read_device_error",
     "q8_version", "q8_packed_bytes", "q8_pack_weights", "q8_unpack_weights", "q8_gemv",
     "q8_gate_up_swiglu", "q8_moe_route", "q8_moe_workspace_bytes", "q8_moe_gemv",
+    "q8_moe_gemv_noalloc",
     "q8_quantize_act", "q8q8_gemv", "q8q8_block_dots",
 ]
 
@@ -47,6 +48,8 @@ _SIGS = {
     "q8_moe_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64, _I64, _I64]),
     "q8_moe_gemv": (_INT, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64,
                            _P, _SZ, _P]),
+    "q8_moe_gemv_noalloc": (_INT, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64,
+                                   _I64, _P]),
     "q8_quantize_act": (_INT, [_P, _P, _P, _I64, _I64, _P]),
     "q8q8_gemv": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "q8q8_block_dots": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
@@ -163,6 +166,13 @@ def q8_moe_gemv(gate_up_experts, down_experts, shared_gate_up, shared_down, idx,
     _call("q8_moe_gemv", _ptr(gate_up_experts), _ptr(down_experts), _ptr(shared_gate_up),
           _ptr(shared_down), _ptr(idx), _ptr(w), _ptr(x), _ptr(y), T, E, top_k, H, I, I_shared,
           _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def q8_moe_gemv_noalloc(gate_up_experts, down_experts, shared_gate_up, shared_down, idx, w, x, y,
+                        T, E, top_k, H, I, I_shared, stream=None):
+    _call("q8_moe_gemv_noalloc", _ptr(gate_up_experts), _ptr(down_experts), _ptr(shared_gate_up),
+          _ptr(shared_down), _ptr(idx), _ptr(w), _ptr(x), _ptr(y), T, E, top_k, H, I, I_shared,
+          _stream(stream))
 
 
 def q8_quantize_act(x, xq, xd, N, K, stream=None):

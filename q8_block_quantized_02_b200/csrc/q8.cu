@@ -293,6 +293,39 @@ static MoePlan plan_moe(int stage, int64_t T, int64_t c_min, int nmax, int64_t u
 
 static size_t moe_hbuf_bytes(int64_t T, int64_t k, int64_t I) { return (size_t)round_up(T * k * I * 4, 256); }
 
+// ---------------------------------------------------------------------------
+// scratch for q8_moe_gemv_noalloc: a fixed array in the library's own device
+// memory, so that call needs no buffer from the caller.  Each device that
+// loads the library holds these bytes until the process exits.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_moe_noalloc_scratch[kNoAllocScratchBytes];
+
+static void *g_moe_noalloc_addr[kMaxDevices];  // device address of the array, per device
+static std::mutex g_moe_noalloc_mutex;
+
+// The array's name is only a host-side stand-in; the address a kernel can use
+// comes from cudaGetSymbolAddress, looked up once per device with that device
+// current (the first call on each device does this).
+static q8_status moe_noalloc_scratch(void **out) {
+    int dev = 0;
+    Q8_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice, "device index");
+    if (!g_moe_noalloc_addr[dev]) {
+        std::lock_guard<std::mutex> lock(g_moe_noalloc_mutex);
+        if (!g_moe_noalloc_addr[dev]) {
+            void *p = nullptr;
+            cudaError_t e = cudaGetSymbolAddress(&p, g_moe_noalloc_scratch);
+            if (e != cudaSuccess || p == nullptr)
+                return cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
+                                 "cudaGetSymbolAddress(moe scratch)");
+            g_moe_noalloc_addr[dev] = p;
+        }
+    }
+    *out = g_moe_noalloc_addr[dev];
+    return Q8_OK;
+}
+
 }  // namespace q8
 
 using namespace q8;
@@ -547,6 +580,28 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
                             "q8_moe_gemv down launch", tq_r, td_r, tq_s, td_s, tx_r, tx_s, a));
     }
     return Q8_OK;
+}
+
+q8_status q8_moe_gemv_noalloc(const void *gate_up_experts, const void *down_experts,
+                              const void *shared_gate_up, const void *shared_down,
+                              const int32_t *idx, const float *w, const float *x, float *y,
+                              int64_t T, int64_t E, int64_t top_k, int64_t H, int64_t I,
+                              int64_t I_shared, q8_stream_t stream) {
+    const size_t need = q8_moe_workspace_bytes(T, E, top_k, H, I, I_shared);
+    if (need == 0) return Q8_ERR_SHAPE;
+    if (need > kNoAllocScratchBytes) {
+        snprintf(last_error_buf(), 256,
+                 "q8_moe_gemv_noalloc: these sizes need %zu bytes of scratch; the built-in "
+                 "scratch holds %zu",
+                 need, kNoAllocScratchBytes);
+        return Q8_ERR_UNSUPPORTED;
+    }
+    void *scratch = nullptr;
+    Q8_CHECK(moe_noalloc_scratch(&scratch));
+    // The MoE launches write every scratch element before they read it, so the
+    // previous call's contents never need clearing.
+    return q8_moe_gemv(gate_up_experts, down_experts, shared_gate_up, shared_down, idx, w, x, y, T,
+                       E, top_k, H, I, I_shared, scratch, need, stream);
 }
 
 }  // extern "C"
