@@ -238,7 +238,11 @@ q8_status q8_quantize_act(const float *x, int8_t *xq, uint16_t *xd, int64_t N, i
  * The int8 x int8 accumulation with the Q8_0 scales of "Add Qwen1.5-MoE Q8_0
  * ... - #144" ("Key implementation notes"), the Q8-native integer dot named
  * as the next step in "Lumen v0.3.0" ("v0.3 -> v0.4 candidate moves").
- * The int32 block dots run on the integer dot-product (dp4a) units.
+ * N <= 4: the int32 block dots run on the integer dot-product (dp4a) units.
+ * 5 <= N <= 16: they run on the tensor cores (tcgen05.mma kind::i8, one
+ * 128 x 16 x 32 MMA per block, activation rows past N read as zero); a launch
+ * with fewer 128-row tiles than SMs splits K over a thread-block cluster of up
+ * to 8 CTAs and adds the partial sums in rank order.  Both are deterministic.
  * W: packed M x K.  xq, xd: as written by q8_quantize_act.  y: [N][M] fp32.
  * fp32 result within 1e-5 * sum_b |d_w d_x| sum_i |q_w q_x| of the exact. */
 q8_status q8q8_gemv(const void *W, const int8_t *xq, const uint16_t *xd, float *y, int64_t M,

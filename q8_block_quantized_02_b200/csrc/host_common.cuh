@@ -210,22 +210,38 @@ inline q8_status encode_map_3d(CUtensorMap *map, CUtensorMapDataType dtype, cons
 // ---------------------------------------------------------------------------
 // launches (programmatic dependent launch on the given stream)
 // ---------------------------------------------------------------------------
+// `cluster_x` > 1 groups consecutive CTAs along x into thread-block clusters.
 template <typename... KArgs, typename... Args>
-inline q8_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                            cudaStream_t stream, const char *name, Args &&...args) {
+inline q8_status launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t stream, const char *name, unsigned cluster_x,
+                                    Args &&...args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int n = 1;
+    if (cluster_x > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = cluster_x;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        n = 2;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = n;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
     if (e != cudaSuccess) return cuda_fail(e, name);
     return Q8_OK;
+}
+
+template <typename... KArgs, typename... Args>
+inline q8_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t stream, const char *name, Args &&...args) {
+    return launch_pdl_cluster(kernel, grid, block, smem, stream, name, 1u, std::forward<Args>(args)...);
 }
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }

@@ -8,6 +8,7 @@
 #include "host_common.cuh"
 #include "pack.cuh"
 #include "q8q8.cuh"
+#include "q8q8_mma.cuh"
 #include "route.cuh"
 #include "tile_gemm.cuh"
 #include "moe.cuh"
@@ -209,6 +210,85 @@ static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, floa
                                              : "q8q8_gemv launch";
     return launch_pdl(k, dim3(p.grid), dim3(p.threads), p.smem, stream, name, tq, td, tq1, td1,
                       tx, a);
+}
+
+// ---------------------------------------------------------------------------
+// Q8 x Q8 on the tensor cores (S8, 9..16 activation columns)
+// ---------------------------------------------------------------------------
+#ifndef Q8_MMA_MIN_N
+#define Q8_MMA_MIN_N 5
+#endif
+constexpr int64_t kMmaMinN = Q8_MMA_MIN_N;  // smallest N sent to the tcgen05 kernel
+constexpr int kMmaMaxStages = 3;
+
+static cudaError_t setup_mma_kernel(int max_smem) {
+    const void *k = reinterpret_cast<const void *>(&q8q8_mma_kernel);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared);
+}
+static RegisterSetup g_reg_mma(setup_mma_kernel);
+
+struct MmaPlan {
+    MmaArgs a;
+    int grid;     // CTAs (a multiple of a.split)
+    size_t smem;
+};
+
+// One CTA per SM.  With at least as many 128-row tiles as SMs each cluster is
+// one CTA walking a contiguous tile range; with fewer, every tile gets a
+// cluster of up to 8 CTAs that split K between them.
+static MmaPlan plan_mma(int64_t M, int64_t K, int64_t N, int sms) {
+    MmaPlan p;
+    MmaArgs &a = p.a;
+    a = MmaArgs{};
+    const int64_t B = K / 32;
+    const int64_t tiles = ceil_div(ceil_div(M, kGroupRows), kMmaTileGroups);
+    int64_t split = 1, clusters = sms;
+    if (tiles < sms) {
+        split = std::min<int64_t>(kMmaMaxSplit, sms / tiles);
+        split = std::min<int64_t>(split, B);  // every CTA keeps at least one block
+        if (split < 1) split = 1;
+        clusters = tiles;
+    }
+    const int64_t blocks = ceil_div(B, split);
+    const int64_t per_cta = ceil_div(tiles, clusters) * ceil_div(blocks, kMmaSB);
+    a.M = (int)M;
+    a.N = (int)N;
+    a.B = (int)B;
+    a.tiles = (int)tiles;
+    a.split = (int)split;
+    a.stages = (int)std::max<int64_t>(1, std::min<int64_t>(kMmaMaxStages, per_cta));
+    p.grid = (int)(clusters * split);
+    p.smem = mma_smem_bytes(a.stages, split > 1);
+    return p;
+}
+
+static q8_status run_mma(const void *W, const int8_t *xq, const uint16_t *xd, float *y, int64_t M,
+                         int64_t K, int64_t N, cudaStream_t stream) {
+    const DeviceInfo *dev = nullptr;
+    Q8_CHECK(device_info(&dev));
+    const int64_t B = K / 32, C = K / 16;
+    const int64_t groups = ceil_div(M, kGroupRows);
+    MmaPlan p = plan_mma(M, K, N, dev->sms);
+    if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
+    p.a.y = y;
+    p.a.xd = xd;
+    const uint64_t gstride = (uint64_t)kGroupBytesPerBlock * B;
+    const uint8_t *dbase = static_cast<const uint8_t *>(W) + 256 * B;
+    CUtensorMap tq, td, tx;
+    // weights: [group][16-byte column][8 rows x 16 B], 16 groups x kMmaCS columns a box
+    Q8_CHECK(make_map_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, kColBytes, C, groups, kColBytes,
+                         gstride, kColBytes, kMmaCS, kMmaTileGroups, true));
+    // scales: [group][block][8 rows] fp16
+    Q8_CHECK(make_map_3d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT16, dbase, 8, B, groups, 16, gstride, 8,
+                         kMmaSB, kMmaTileGroups, true));
+    // activations: [16-byte column][row][16 B]; rows past N read as zero
+    Q8_CHECK(make_map_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, 16, N, C, (uint64_t)K, 16, 16,
+                         kMmaN, kMmaCS, false));
+    return launch_pdl_cluster(q8q8_mma_kernel, dim3(p.grid), dim3(kMmaThreads), p.smem, stream,
+                              "q8q8_gemv (tensor cores) launch", (unsigned)p.a.split, tq, td, tx, p.a);
 }
 
 // ---------------------------------------------------------------------------
@@ -440,6 +520,7 @@ q8_status q8q8_gemv(const void *W, const int8_t *xq, const uint16_t *xd, float *
     Q8_CHECK(check_device_ptr(xd, false));
     if (reinterpret_cast<uintptr_t>(xd) & 1u) return Q8_ERR_ALIGN;
     Q8_CHECK(check_device_ptr(y));
+    if (N >= kMmaMinN) return run_mma(W, xq, xd, y, M, K, N, (cudaStream_t)stream);
     return run_tile(W, xq, xd, y, M, K, N, kModeQ8Q8, (cudaStream_t)stream);
 }
 

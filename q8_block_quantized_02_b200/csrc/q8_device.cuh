@@ -25,6 +25,7 @@ enum : unsigned int {
     kErrWaitTimeout = 1u << 0,   // a pipeline barrier wait ran past its limit
     kErrDrainTimeout = 1u << 1,  // waiting for in-flight copies at exit ran out
     kErrBadExpert = 1u << 2,     // an expert index outside [0, E) was seen
+    kErrLaunchConfig = 1u << 3,  // shared memory, cluster or tensor memory differ from the plan
 };
 
 __device__ unsigned int g_q8_error;
@@ -81,6 +82,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait that may suspend the thread for up to `hint_ns` while the phase is
+// incomplete, so a waiting thread takes no issue slots from working warps.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Suspend-time hint of the waiting loops: far below the wait limit, so the
+// limit and the abort flag are still checked often.
+constexpr uint32_t kWaitHintNs = 20000;
+
 // Wait for the phase with the given parity to complete.  Returns false (and
 // raises *abort) when the wait runs past kWaitLimitNs; returns false at once
 // when *abort is already raised, so that every thread of a CTA leaves a broken
@@ -89,17 +108,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     if (abort && *abort) return false;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0) {
-            if (abort && *abort) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                record_error(kErrWaitTimeout);
-                if (abort) *abort = 1;
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
+        if (abort && *abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_error(kErrWaitTimeout);
+            if (abort) *abort = 1;
+            return false;
         }
     }
+}
+
+// mbar_wait for a whole warp: lane 0 alone polls the barrier (32 lanes polling
+// one barrier serialise in the shared-memory pipe), then __syncwarp orders its
+// acquire before every lane's reads of the guarded data.  Warp-uniform result.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
+    __syncwarp();
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 // Bounded wait used while draining in-flight copies before a CTA exits.

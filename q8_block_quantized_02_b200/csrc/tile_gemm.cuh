@@ -422,7 +422,15 @@ __global__ void __launch_bounds__(ColsCfg<NMAX, MODE, CW_>::THREADS, 1)
             for (int ks = 0; ks < a.ksteps; ++ks, ++it) {
                 if (it % Cfg::GROUPS != cg) continue;
                 const int slot = it % a.stages;
-                if (mbar_wait(full0 + 8 * slot, (it / a.stages) & 1, abort_flag)) {
+                // With two groups a slot can pass from one group to the other
+                // (odd ring): wait for the release of the slot's previous
+                // stage, as the producer does, before waiting for this fill.
+                // Otherwise, while that stage is still in flight, the previous
+                // phase of `full` has the parity this wait asks for.
+                bool ready = true;
+                if (Cfg::GROUPS > 1 && it >= a.stages)
+                    ready = mbar_wait(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag);
+                if (ready && mbar_wait(full0 + 8 * slot, (it / a.stages) & 1, abort_flag)) {
                     const uint8_t *st = smem + (size_t)slot * a.stage_bytes;
                     const int cols = min(a.CS, a.C - ks * a.CS);
                     const int nq = (cols + 3) >> 2;

@@ -107,6 +107,52 @@ def test_q8q8_ragged_shapes(M, K, N):
     assert_within(y, y_ref, TOL_REL * y_abs, f"q8q8 {M}x{K} N={N}")
 
 
+@pytest.mark.parametrize("M,K,N", [
+    (4096, 896, 9),        # K split over a cluster of 4, one stage per CTA
+    (4096, 3584, 12),      # cluster of 4, pipelined stages
+    (1000, 2048, 13),      # ragged last tile (125 groups)
+    (136, 96, 16),         # 17 groups: a tile of 16 and a tile of 1; 3 blocks over 3 CTAs
+    (896, 896, 16),        # cluster of 8, 3-4 blocks per CTA (partial stage)
+    (3584, 18944, 16),     # cluster of 5 with uneven K slices
+    (37888, 3584, 16),     # one CTA per SM walking two tiles
+    (151936, 896, 16),     # 1187 tiles: the vocabulary projection
+])
+def test_q8q8_tensor_core_shapes(M, K, N):
+    """N >= 9 runs on the tcgen05 kernel: 128-row tiles, K split across a
+    cluster when there are fewer tiles than SMs."""
+    g, x = q8gen.q8_matrix(M + 7 * K + N, M, K, N)
+    xq, xd, _ = oracle.quantize_act(x)
+    y = run_q8q8(g, xq, xd, M, K)
+    assert np.all(np.isfinite(y))
+    if M * K <= 4096 * 3584:
+        rows = np.arange(M)
+    else:
+        rng = np.random.default_rng(M + K)
+        rows = np.unique(np.concatenate([rng.integers(0, M, 384), np.arange(128), np.arange(M - 136, M)]))
+    _, y_ref, y_abs = oracle.q8q8(rows_subset(g, M, K, rows), xq, xd, len(rows), K, want_dots=False,
+                                  threads=oracle.max_threads())
+    assert_within(y[:, rows], y_ref, TOL_REL * y_abs, f"q8q8 tensor cores {M}x{K} N={N}")
+
+
+def test_q8q8_tensor_core_deterministic_and_exact_on_integers():
+    """Run-to-run identical; with unit scales every output is an exact integer
+    sum of block dots, so the result must equal the oracle's exactly."""
+    M, K, N = 4096, 3584, 16
+    g, x = q8gen.q8_matrix(5, M, K, N)
+    xq, xd, _ = oracle.quantize_act(x)
+    y1 = run_q8q8(g, xq, xd, M, K)
+    y2 = run_q8q8(g, xq, xd, M, K)
+    assert np.array_equal(y1, y2)
+    # scales of exactly 1.0 (binary16 0x3C00): y = sum of int32 block dots,
+    # which fp32 holds exactly while |partial sums| < 2^24
+    qw, _ = q8gen.split_gguf(g, M, K)
+    g1 = q8gen.assemble_gguf(qw, np.full((M, K // 32), 0x3C00, np.uint16))
+    xd1 = np.full_like(xd, 0x3C00)
+    y = run_q8q8(g1, xq, xd1, M, K)
+    dots, y_ref, _ = oracle.q8q8(g1, xq, xd1, M, K, threads=oracle.max_threads())
+    assert np.array_equal(y.astype(np.float64), y_ref)
+
+
 def test_quantize_then_q8q8_end_to_end():
     """GPU quantiser feeding the GPU product equals the oracle chain."""
     M, K, N = 4096, 3584, 16
