@@ -171,6 +171,106 @@ static TilePlan plan_tile(int64_t units, int64_t C, int64_t N, int mode, int sms
     return p;
 }
 
+// ---------------------------------------------------------------------------
+// resident kernel: small matrices whose CTA-share of weights fits in shared
+// memory (see tile_gemm.cuh)
+// ---------------------------------------------------------------------------
+using ResidentKernel = void (*)(CUtensorMap, CUtensorMap, const float *, TileArgs);
+
+// N = 1 only: a CTA of this kernel leaves most of the SM's registers to the
+// next kernel on the stream (wider N would take them all).
+static ResidentKernel resident_kernel_for(int mode) {
+    return mode == kModeSwiGLU ? &resident_kernel<1, kModeSwiGLU> : &resident_kernel<1, kModeF32>;
+}
+static int resident_red_floats(int mode) {
+    return mode == kModeSwiGLU ? res_red_floats<1, kModeSwiGLU>() : res_red_floats<1, kModeF32>();
+}
+
+static cudaError_t setup_resident_kernels(int max_smem) {
+    for (int mode = 0; mode < 2; ++mode) {
+        const void *k = reinterpret_cast<const void *>(resident_kernel_for(mode));
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+static RegisterSetup g_reg_resident(setup_resident_kernels);
+
+// Shared memory a resident launch may take: room is left on the SM for the
+// next kernel on the stream to become resident early.
+constexpr int64_t kResidentSmemBudget = 100 * 1024;
+
+// Plan for the resident kernel, or false when the matrix is too large for it
+// (more than kResTGM row groups per CTA, or the weights do not fit).
+static bool plan_resident(int64_t units, int64_t C, int64_t N, int mode, int sms, TilePlan *out) {
+    if (mode != kModeF32 && mode != kModeSwiGLU) return false;
+    if (N != 1) return false;
+    const int64_t grid = units < sms ? units : sms;
+    const int64_t upc = ceil_div(units, grid);
+    if (upc > kResTGM) return false;
+    const int64_t halves = mode == kModeSwiGLU ? 2 : 1;
+    // weight boxes of at most 256 columns, as even as multiples of 16 allow
+    const int64_t nchunks = ceil_div(C, 256);
+    const int64_t cb = round_up(ceil_div(C, nchunks), 16);
+    const int64_t cs = nchunks * cb;
+    TilePlan p;
+    TileArgs &a = p.a;
+    a = TileArgs{};
+    a.N = (int)N;
+    a.C = (int)C;
+    a.B = (int)(C / 2);
+    a.units = (int)units;
+    a.TG = (int)upc;
+    a.CS = (int)cs;
+    a.ksteps = 1;
+    a.NQ = (int)ceil_div(C, 4);
+    a.stages = 1;
+    a.CB = (int)cb;
+    a.nchunks = (int)nchunks;
+    a.q_box = (uint32_t)(cs * kColBytes);
+    a.d_box = (uint32_t)(cs * 8);
+    a.d_slot = a.d_box;
+    a.x_box = (uint32_t)(N * cs * 64);
+    a.q_half = (uint32_t)(upc * a.q_box);
+    a.d_off = (uint32_t)(halves * a.q_half);
+    a.d_half = (uint32_t)(upc * a.d_box);
+    a.x_off = a.d_off + (uint32_t)(halves * a.d_half);
+    a.stage_bytes = (uint32_t)round_up(a.x_off + a.x_box, 128);
+    const int64_t smem = (int64_t)a.stage_bytes + (int64_t)resident_red_floats(mode) * 4 + 16;
+    if (smem > kResidentSmemBudget) return false;
+    if (halves * upc * (int64_t)(a.q_box + a.d_box) >= (1 << 20)) return false;  // mbarrier tx count
+    p.grid = (int)grid;
+    p.threads = kResThreads;
+    p.wide = false;
+    p.smem = (size_t)smem;
+    *out = p;
+    return true;
+}
+
+static q8_status run_resident(const TilePlan &plan, const void *W, const float *x, float *y,
+                              int64_t rows_out, int64_t K, int64_t N, int mode, cudaStream_t stream) {
+    TilePlan p = plan;
+    TileArgs &a = p.a;
+    const bool swiglu = mode == kModeSwiGLU;
+    const int64_t B = K / 32, C = K / 16;
+    const int64_t total_groups = swiglu ? 2 * (int64_t)a.units : a.units;
+    a.y = y;
+    a.M_out = (int)rows_out;
+    a.up_group0 = swiglu ? a.units : 0;
+    const uint64_t gstride = (uint64_t)kGroupBytesPerBlock * B;
+    const uint8_t *dbase = static_cast<const uint8_t *>(W) + 256 * B;
+    CUtensorMap tq, td;
+    Q8_CHECK(make_map_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, kColBytes, C, total_groups, kColBytes,
+                         gstride, kColBytes, a.CB, 1, true));
+    Q8_CHECK(make_map_3d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT16, dbase, 8, B, total_groups, 16, gstride, 8,
+                         a.CB / 2, 1, true));
+    return launch_pdl(resident_kernel_for(mode), dim3(p.grid), dim3(p.threads), p.smem, stream,
+                      swiglu ? "q8_gate_up_swiglu launch" : "q8_gemv launch", tq, td, x, a);
+}
+
 static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, float *y,
                           int64_t rows_out, int64_t K, int64_t N, int mode, cudaStream_t stream) {
     const bool swiglu = mode == kModeSwiGLU;
@@ -179,6 +279,12 @@ static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, floa
     const int64_t B = K / 32, C = K / 16;
     const int64_t units = ceil_div(rows_out, kGroupRows);
     const int64_t total_groups = swiglu ? 2 * units : units;
+    {
+        TilePlan rp;
+        if (plan_resident(units, C, N, mode, dev->sms, &rp) && rp.smem <= (size_t)dev->max_smem_optin &&
+            (uint64_t)units * (uint64_t)rp.grid < (1ull << 31))
+            return run_resident(rp, W, static_cast<const float *>(x), y, rows_out, K, N, mode, stream);
+    }
     TilePlan p = plan_tile(units, C, N, mode, dev->sms);
     TileArgs &a = p.a;
     a.y = y;

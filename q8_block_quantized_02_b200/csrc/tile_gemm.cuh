@@ -63,6 +63,8 @@ struct TileArgs {
     uint32_t d_half;     // TG * d_slot
     uint32_t x_off;      // offset of the activation region
     uint32_t stage_bytes;
+    int CB;              // resident kernel: columns per weight box
+    int nchunks;         // resident kernel: weight boxes per row group (CS = nchunks * CB)
 };
 
 template <int MODE>
@@ -472,6 +474,154 @@ __global__ void __launch_bounds__(ColsCfg<NMAX, MODE, CW_>::THREADS, 1)
     }
     __syncthreads();
     if (threadIdx.x == 0 && *abort_flag) tile_drain(full0, a, *issued);
+}
+
+// ---------------------------------------------------------------------------
+// Resident kernel (small matrices, N <= 4)
+// ---------------------------------------------------------------------------
+// For matrices whose row groups spread to at most 8 per CTA, with all of a
+// CTA's weights fitting in shared memory (the decode projections of small
+// models).  Every weight box of the CTA is issued at kernel start, before
+// griddepcontrol.wait, so the weights stream in while the previous kernel on
+// the stream still runs.  After the wait the activations are copied with
+// plain 16-byte loads (one L2 round trip), the CTA computes all of its rows
+// from shared memory in one pass with the column-owner lane mapping above,
+// and the eight warps' partial sums meet in shared memory behind a single
+// barrier, added in warp order.  There is no ring, no per-stage barrier and
+// no reducer warp: a dependent decode step pays for none of them.
+constexpr int kResWarps = 8;
+constexpr int kResThreads = kResWarps * 32;
+constexpr int kResTGM = 8;   // row groups per CTA at most
+
+template <int NMAX, int MODE>
+__host__ __device__ constexpr int res_red_floats() {
+    return kResWarps * kResTGM * (MODE == kModeSwiGLU ? 2 : 1) * NMAX * 8;
+}
+
+template <int NMAX, int MODE>
+__global__ void __launch_bounds__(kResThreads, 1)
+    resident_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap td,
+                    const float *__restrict__ x, const TileArgs a) {
+    constexpr int H = MODE == kModeSwiGLU ? 2 : 1;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float *red = reinterpret_cast<float *>(smem + a.stage_bytes);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(red + res_red_floats<NMAX, MODE>());
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bar + 1);
+    const uint32_t wbar = smem_u32(bar);
+    // units * grid < 2^31 is checked on the host, so 32-bit math is exact here
+    const int u0 = (int)(((unsigned)a.units * blockIdx.x) / gridDim.x);
+    const int u1 = (int)(((unsigned)a.units * (blockIdx.x + 1)) / gridDim.x);
+    const int tga = u1 - u0;  // <= kResTGM (planned on the host)
+    if (threadIdx.x == 0) {
+        mbar_init(wbar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // The next kernel on the stream may start its prologue now; it reads
+    // nothing this kernel writes before its own griddepcontrol.wait.
+    pdl_launch_dependents();
+    if (threadIdx.x == 0) {
+        const uint64_t pw = policy_evict_first();
+        const uint32_t st = smem_u32(smem);
+        mbar_arrive_expect_tx(wbar, (uint32_t)(H * tga) * (a.q_box + a.d_box));
+        for (int h = 0; h < H; ++h)
+            for (int g = 0; g < tga; ++g) {
+                const int grp = u0 + g + (h ? a.up_group0 : 0);
+                for (int c = 0; c < a.nchunks; ++c) {
+                    tma_load_3d(st + h * a.q_half + g * a.q_box + c * a.CB * kColBytes, &tq, wbar, 0,
+                                c * a.CB, grp, pw);
+                    tma_load_3d(st + a.d_off + h * a.d_half + g * a.d_slot + c * a.CB * 8, &td, wbar, 0,
+                                c * a.CB / 2, grp, pw);
+                }
+            }
+    }
+    pdl_wait();  // the activations, and the outputs, belong to the previous grid until here
+    {
+        // activations -> shared memory as [n][column][16 floats]; every load of a
+        // thread is issued before its first store, so the copy costs one round trip
+        constexpr int XB = 8;
+        const int k4 = a.C * 4;  // float4 per activation row
+        const int total = a.N * k4;
+        float4 *xs = reinterpret_cast<float4 *>(smem + a.x_off);
+        const float4 *xg = reinterpret_cast<const float4 *>(x);
+        for (int base = threadIdx.x; base < total; base += XB * kResThreads) {
+            float4 v[XB];
+#pragma unroll
+            for (int u = 0; u < XB; ++u) {
+                const int i = base + u * kResThreads;
+                if (i < total) v[u] = __ldg(xg + i);
+            }
+#pragma unroll
+            for (int u = 0; u < XB; ++u) {
+                const int i = base + u * kResThreads;
+                if (i < total) {
+                    const int n = i / k4;
+                    xs[n * a.CS * 4 + (i - n * k4)] = v[u];
+                }
+            }
+        }
+    }
+    __syncthreads();
+    const bool ok = mbar_wait_warp(wbar, 0, abort_flag);
+    const int r = lane & 7, j = lane >> 3;
+    float acc[kResTGM][H][NMAX];
+#pragma unroll
+    for (int g = 0; g < kResTGM; ++g)
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+#pragma unroll
+            for (int n = 0; n < NMAX; ++n) acc[g][h][n] = 0.f;
+    if (ok) {
+        const int nq = (a.C + 3) >> 2;
+        for (int cq = warp; cq < nq; cq += kResWarps) {
+            const int col = 4 * cq + j;
+            if (tga == kResTGM)
+                cols_step<NMAX, MODE, kResTGM, false>(smem, a, 0, col, a.C, r, j, tga, acc);
+            else
+                cols_step<NMAX, MODE, kResTGM, true>(smem, a, 0, col, a.C, r, j, tga, acc);
+        }
+    }
+    // lanes r, r+8, r+16, r+24 hold partial sums of the same row
+#pragma unroll
+    for (int g = 0; g < kResTGM; ++g)
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+#pragma unroll
+            for (int n = 0; n < NMAX; ++n) {
+                acc[g][h][n] += __shfl_xor_sync(0xffffffffu, acc[g][h][n], 8);
+                acc[g][h][n] += __shfl_xor_sync(0xffffffffu, acc[g][h][n], 16);
+            }
+    if (j == 0) {
+#pragma unroll
+        for (int g = 0; g < kResTGM; ++g)
+#pragma unroll
+            for (int h = 0; h < H; ++h)
+#pragma unroll
+                for (int n = 0; n < NMAX; ++n)
+                    red[((((warp * kResTGM + g) * H + h) * NMAX + n) << 3) + r] = acc[g][h][n];
+    }
+    __syncthreads();
+    if (ok) {
+        for (int o = threadIdx.x; o < tga * 8; o += kResThreads) {
+            const int g = o >> 3, rr = o & 7;
+            float v[H][NMAX];
+#pragma unroll
+            for (int h = 0; h < H; ++h)
+#pragma unroll
+                for (int n = 0; n < NMAX; ++n) {
+                    float sum = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kResWarps; ++w)
+                        sum += red[((((w * kResTGM + g) * H + h) * NMAX + n) << 3) + rr];
+                    v[h][n] = sum;
+                }
+            store_unit<NMAX, MODE>(a, u0 + g, rr, v[0], v[H - 1]);
+        }
+    } else if (threadIdx.x == 0) {
+        mbar_drain(wbar, 0);  // no weight copy may still land after the CTA exits
+    }
 }
 
 // ---------------------------------------------------------------------------

@@ -1,0 +1,107 @@
+"""Run one libq8 product on synthetic Qwen-shaped inputs and time it.
+
+    python -m q8_block_quantized_02_b200.profile --op gemv --M 151936 --K 896 --N 1
+    python -m q8_block_quantized_02_b200.profile --op q8q8 --M 37888 --K 3584 --N 16
+
+Weights follow the synthetic Q8_0 recipe (q uniform in [-127, 127], d =
+|N(0,1)| * 0.02) and activations are N(0,1).  Enough packed copies of the
+weight matrix are made to cover three times the L2 cache, and the calls walk
+through them, so every timed call streams its weights from HBM.  Each call is
+one launch of the library's kernel on the current stream; the time per call
+comes from CUDA events around `--reps` back-to-back calls after `--warmup`
+untimed ones.  Prints one JSON line with microseconds per call and the weight
+bytes (34 per 32 weights) per second.
+
+This is also the driver for ncu captures of a single kernel: with
+`--copies 1 --reps 3 --warmup 2` it makes five launches on one matrix.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--op", choices=["gemv", "swiglu", "q8q8"], default="gemv",
+                    help="q8_gemv, q8_gate_up_swiglu (M = rows of the stacked gate|up matrix) "
+                         "or q8_quantize_act + q8q8_gemv (only q8q8_gemv is timed)")
+    ap.add_argument("--M", type=int, default=151936)
+    ap.add_argument("--K", type=int, default=896)
+    ap.add_argument("--N", type=int, default=1)
+    ap.add_argument("--reps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--copies", type=int, default=0, help="packed weight copies (0: cover 3x L2)")
+    ap.add_argument("--seed", type=int, default=0)
+    args = ap.parse_args(argv)
+
+    import numpy as np
+    import torch
+
+    import q8gen
+    import q8_block_quantized_02_b200 as q8
+
+    M, K, N = args.M, args.K, args.N
+    dev = torch.device("cuda", torch.cuda.current_device())
+    g, x = q8gen.q8_matrix(args.seed, M, K, N)
+    nbytes = q8.q8_packed_bytes(M, K)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = args.copies if args.copies > 0 else max(1, int(np.ceil(3 * l2 / nbytes)))
+    src = torch.from_numpy(g).to(dev)
+    packs = []
+    for _ in range(copies):
+        p = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        q8.q8_pack_weights(src, M, K, p)
+        packs.append(p)
+    del src
+    xf = torch.from_numpy(x).to(dev)
+    if args.op == "swiglu":
+        if M % 16:
+            raise SystemExit("--op swiglu needs M = 2 * I with I % 8 == 0")
+        y = torch.empty((N, M // 2), dtype=torch.float32, device=dev)
+    else:
+        y = torch.empty((N, M), dtype=torch.float32, device=dev)
+    if args.op == "q8q8":
+        xq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        xd = torch.empty((N, K // 32), dtype=torch.int16, device=dev)
+        q8.q8_quantize_act(xf, xq, xd, N, K)
+
+    it = [0]
+
+    def call():
+        p = packs[it[0] % copies]
+        it[0] += 1
+        if args.op == "gemv":
+            q8.q8_gemv(p, xf, y, M, K, N)
+        elif args.op == "swiglu":
+            q8.q8_gate_up_swiglu(p, xf, y, M // 2, K, N)
+        else:
+            q8.q8q8_gemv(p, xq, xd, y, M, K, N)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.reps):
+        call()
+    t1.record()
+    torch.cuda.synchronize()
+    st, word = q8.q8_read_device_error()
+    us = t0.elapsed_time(t1) * 1e3 / max(1, args.reps)
+    weight_bytes = M * K * 34 // 32
+    print(json.dumps({"op": args.op, "M": M, "K": K, "N": N, "us_per_call": round(us, 3),
+                      "weight_GBps": round(weight_bytes / (us * 1e-6) / 1e9, 1), "copies": copies,
+                      "reps": args.reps, "device_error": word}), flush=True)
+    return 0 if st == 0 else 1
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())
