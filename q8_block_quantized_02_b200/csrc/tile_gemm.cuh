@@ -493,9 +493,78 @@ constexpr int kResWarps = 8;
 constexpr int kResThreads = kResWarps * 32;
 constexpr int kResTGM = 8;   // row groups per CTA at most
 
+constexpr int kResColsPerThread = 2;  // one-group path: C <= 512 columns
+
 template <int NMAX, int MODE>
 __host__ __device__ constexpr int res_red_floats() {
-    return kResWarps * kResTGM * (MODE == kModeSwiGLU ? 2 : 1) * NMAX * 8;
+    // column-owner partials, or the one-group path's [row][thread] partials
+    return kResWarps * kResTGM * (MODE == kModeSwiGLU ? 2 : 1) * NMAX * 8 > 8 * kResThreads
+               ? kResWarps * kResTGM * (MODE == kModeSwiGLU ? 2 : 1) * NMAX * 8
+               : 8 * kResThreads;
+}
+
+// One row group, fp32 activations, N = 1: thread t owns the 16-byte columns
+// t and t + 256 of the group.  It loads their activations straight from
+// memory, reads each column's 8 x 16 B core matrix a row at a time starting at
+// row t % 8 (the eight lanes of a quarter-warp then read eight different
+// 16-byte bank groups), and keeps one partial sum per row, in that rotated
+// order.  Partials meet in shared memory as [row][thread]; warp r adds row
+// r's in thread order and then across its lanes by a fixed shuffle tree.
+// With a single row group per CTA the column-owner mapping would have eight
+// lanes read every activation; here each is read once.  (With several
+// groups or the SwiGLU pair the column-owner mapping reuses the activations
+// across groups and stays faster.)
+__device__ __forceinline__ void res_one_group(const uint8_t *smem, const TileArgs &a,
+                                              const float *__restrict__ x, int unit, uint32_t wbar,
+                                              volatile int *abort_flag, float *red) {
+    const int t = threadIdx.x, rot = t & 7, lane = t & 31, warp = t >> 5;
+    ulonglong2 xa[kResColsPerThread][4];
+#pragma unroll
+    for (int k = 0; k < kResColsPerThread; ++k) {
+        const int c = t + k * kResThreads;
+        if (c < a.C) {
+            const ulonglong2 *xg = reinterpret_cast<const ulonglong2 *>(x + (size_t)c * 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xa[k][i] = __ldg(xg + i);
+        }
+    }
+    const bool ok = mbar_wait_warp(wbar, 0, abort_flag);
+    float accr[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) accr[i] = 0.f;
+    if (ok) {
+#pragma unroll
+        for (int k = 0; k < kResColsPerThread; ++k) {
+            const int c = t + k * kResThreads;
+            if (c < a.C) {
+                const uint8_t *qc = smem + c * kColBytes;
+                const uint8_t *dc = smem + a.d_off + (c >> 1) * 16;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = (i + rot) & 7;
+                    const uint4 qv = *reinterpret_cast<const uint4 *>(qc + r * 16);
+                    const float d = __half2float(*reinterpret_cast<const __half *>(dc + r * 2));
+                    uint64_t w[8];
+                    dequant16_x2(qv, w);
+                    accr[i] = fmaf(dot16_x2(w, xa[k][0], xa[k][1], xa[k][2], xa[k][3]), d, accr[i]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[((i + rot) & 7) * kResThreads + t] = accr[i];
+    __syncthreads();
+    if (ok && warp < 8) {
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < kResThreads / 32; ++i) sum += red[warp * kResThreads + lane + 32 * i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) {
+            const int row = unit * kGroupRows + warp;
+            if (row < a.M_out) a.y[row] = sum;
+        }
+    }
 }
 
 template <int NMAX, int MODE>
@@ -538,6 +607,11 @@ __global__ void __launch_bounds__(kResThreads, 1)
             }
     }
     pdl_wait();  // the activations, and the outputs, belong to the previous grid until here
+    if (MODE == kModeF32 && NMAX == 1 && tga == 1 && a.C <= kResColsPerThread * kResThreads) {
+        res_one_group(smem, a, x, u0, wbar, abort_flag, red);
+        if (threadIdx.x == 0 && *abort_flag) mbar_drain(wbar, 0);
+        return;
+    }
     {
         // activations -> shared memory as [n][column][16 floats]; every load of a
         // thread is issued before its first store, so the copy costs one round trip
