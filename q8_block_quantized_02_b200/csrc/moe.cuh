@@ -212,8 +212,7 @@ __global__ void __launch_bounds__(kMoeThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(red + RED);
     volatile int *issued = abort_flag + 1;
 
-    pdl_launch_dependents();
-    pdl_wait();  // idx, w (router) and the activations come from earlier kernels
+    pdl_wait_and_trigger();  // idx, w (router) and the activations come from earlier kernels
     moe_build_table(tb, a, STAGE);
 
     // this CTA's range of units

@@ -178,17 +178,31 @@ static TilePlan plan_tile(int64_t units, int64_t C, int64_t N, int mode, int sms
 using ResidentKernel = void (*)(CUtensorMap, CUtensorMap, const float *, TileArgs);
 
 // N = 1 only: a CTA of this kernel leaves most of the SM's registers to the
-// next kernel on the stream (wider N would take them all).
-static ResidentKernel resident_kernel_for(int mode) {
-    return mode == kModeSwiGLU ? &resident_kernel<1, kModeSwiGLU> : &resident_kernel<1, kModeF32>;
+// next kernel on the stream (wider N would take them all).  One instance per
+// row-group count, so the column step needs no per-group branch.
+template <int MODE>
+static ResidentKernel resident_kernel_mode(int tgm) {
+    switch (tgm) {
+        case 1: return &resident_kernel<1, MODE, 1>;
+        case 2: return &resident_kernel<1, MODE, 2>;
+        case 3: return &resident_kernel<1, MODE, 3>;
+        case 4: return &resident_kernel<1, MODE, 4>;
+        case 5: return &resident_kernel<1, MODE, 5>;
+        case 6: return &resident_kernel<1, MODE, 6>;
+        case 7: return &resident_kernel<1, MODE, 7>;
+        default: return &resident_kernel<1, MODE, 8>;
+    }
+}
+static ResidentKernel resident_kernel_for(int mode, int tgm) {
+    return mode == kModeSwiGLU ? resident_kernel_mode<kModeSwiGLU>(tgm) : resident_kernel_mode<kModeF32>(tgm);
 }
 static int resident_red_floats(int mode) {
     return mode == kModeSwiGLU ? res_red_floats<1, kModeSwiGLU>() : res_red_floats<1, kModeF32>();
 }
 
 static cudaError_t setup_resident_kernels(int max_smem) {
-    for (int mode = 0; mode < 2; ++mode) {
-        const void *k = reinterpret_cast<const void *>(resident_kernel_for(mode));
+    for (int i = 0; i < 2 * kResTGM; ++i) {
+        const void *k = reinterpret_cast<const void *>(resident_kernel_for(i / kResTGM, 1 + i % kResTGM));
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -267,7 +281,7 @@ static q8_status run_resident(const TilePlan &plan, const void *W, const float *
                          gstride, kColBytes, a.CB, 1, true));
     Q8_CHECK(make_map_3d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT16, dbase, 8, B, total_groups, 16, gstride, 8,
                          a.CB / 2, 1, true));
-    return launch_pdl(resident_kernel_for(mode), dim3(p.grid), dim3(p.threads), p.smem, stream,
+    return launch_pdl(resident_kernel_for(mode, a.TG), dim3(p.grid), dim3(p.threads), p.smem, stream,
                       swiglu ? "q8_gate_up_swiglu launch" : "q8_gemv launch", tq, td, x, a);
 }
 

@@ -174,6 +174,14 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// The kernels trigger their dependents only once their own wait has returned
+// (every thread, after its wait): then at most the next kernel on the stream
+// is resident early, prefetching its weights, and the block scheduler keeps
+// free SMs, so two CTAs of one kernel seldom share an SM.
+__device__ __forceinline__ void pdl_wait_and_trigger() {
+    pdl_wait();
+    pdl_launch_dependents();
+}
 
 // Named barrier over `threads` threads (a multiple of 32).
 __device__ __forceinline__ void named_barrier(int id, int threads) {

@@ -297,9 +297,6 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         n_tiles = 0;
     }
     const int total = n_tiles * ksteps;
-    // The next kernel on the stream may start its prologue; it reads nothing
-    // this kernel writes before its own griddepcontrol.wait.
-    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------ producer ------------------------------
@@ -324,7 +321,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
             const int pro = total < a.stages ? total : a.stages;
             int it = 0;
             for (; it < pro; ++it) issue_w(it);  // weights never depend on the previous grid
-            pdl_wait();                          // activations may
+            pdl_wait_and_trigger();              // activations may
             for (int k = 0; k < pro; ++k) issue_x(k);
             for (; it < total; ++it) {
                 const int slot = it % a.stages;
@@ -333,9 +330,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                 issue_x(it);
             }
             *issued = it;
+        } else {
+            pdl_wait_and_trigger();
         }
     } else if (warp == 1) {
         // ------------------------------ MMA issuer ----------------------------
+        pdl_wait_and_trigger();  // its inputs arrive after the producer's wait anyway
         if (lane == 0) {
             // Block j of every stage goes to TMEM columns 16 j; the two halves
             // (blocks 0-3, 4-7) are each handed to the epilogue by one commit.
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         const bool tab_thread = e < kMmaSB * kMmaN;
         const int jt = (e >> 4) & (kMmaSB - 1), nt = e & 15;  // (block in stage, activation row)
         const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + n0;
-        pdl_wait();  // activation scales and outputs belong to the previous grid until now
+        pdl_wait_and_trigger();  // activation scales and outputs belong to the previous grid until now
         auto dx_load = [&](int it) -> float {
             if (it >= total || !tab_thread) return 0.f;
             const int b = b_lo + (it % ksteps) * kMmaSB + jt;

@@ -222,7 +222,7 @@ __device__ __forceinline__ void tile_produce(uint8_t *smem, uint32_t full0, uint
     const int pro = total < a.stages ? total : a.stages;
     int it = 0;
     for (; it < pro; ++it) issue_weights(it);  // weights never depend on the previous grid
-    pdl_wait();                                // activations may
+    pdl_wait_and_trigger();                    // activations may
     for (int k = 0; k < pro; ++k) issue_x(k);
     for (; it < total; ++it) {
         const int slot = it % a.stages;
@@ -370,17 +370,16 @@ __global__ void __launch_bounds__(ColsCfg<NMAX, MODE, CW_>::THREADS, 1)
         fence_mbar_init();
     }
     __syncthreads();
-    // The next kernel on the stream may start its prologue now; it reads
-    // nothing this kernel writes before its own griddepcontrol.wait.
-    pdl_launch_dependents();
 
     if (warp == CW) {
         if (lane == 0)
             tile_produce<MODE>(smem, full0, empty0, abort_flag, issued, a, u0, u1, total, &tq, &td,
                                &tq1, &td1, &tx);
+        else
+            pdl_wait_and_trigger();
     } else if (warp == CW + 1) {
         // ------------------------------ reducer -------------------------------
-        pdl_wait();  // the outputs may still be read by the previous grid
+        pdl_wait_and_trigger();  // the outputs may still be read by the previous grid
         for (int tl = 0; tl < n_tiles; ++tl) {
             const int p = tl & 1;
             const bool ok = mbar_wait(redfull0 + 8 * p, (tl >> 1) & 1, abort_flag);
@@ -409,7 +408,7 @@ __global__ void __launch_bounds__(ColsCfg<NMAX, MODE, CW_>::THREADS, 1)
     } else {
         // ------------------------------ consumers -----------------------------
         const int cw = warp, cg = cw / WPG, lw = cw % WPG, r = lane & 7, j = lane >> 3;
-        if (MODE == kModeQ8Q8) pdl_wait();  // activation scales are read straight from memory
+        pdl_wait_and_trigger();  // Q8Q8: activation scales are read straight from memory
         int it = 0;
         for (int tl = 0; tl < n_tiles; ++tl) {
             const int ut = u0 + tl * a.TG;
@@ -567,7 +566,43 @@ __device__ __forceinline__ void res_one_group(const uint8_t *smem, const TileArg
     }
 }
 
-template <int NMAX, int MODE>
+// One column of the CTA's TGM row groups for lane (r, j), with no per-group
+// branch so that the groups' independent chains (shared loads,
+// dequantisation, dot products) overlap.  A CTA holding fewer groups (tga <
+// TGM) reads its last group again in place of each missing one; those sums
+// are never stored.
+template <int NMAX, int MODE, int TGM>
+__device__ __forceinline__ void res_step(const uint8_t *st, const TileArgs &a, int col, int r, int tga,
+                                         float (&acc)[TGM][MODE == kModeSwiGLU ? 2 : 1][NMAX]) {
+    constexpr int H = MODE == kModeSwiGLU ? 2 : 1;
+    ulonglong2 xr[NMAX][4];
+#pragma unroll
+    for (int n = 0; n < NMAX; ++n) {
+        if (n < a.N) {
+            const ulonglong2 *xv = reinterpret_cast<const ulonglong2 *>(st + a.x_off + (n * a.CS + col) * 64);
+            xr[n][0] = xv[0];
+            xr[n][1] = xv[1];
+            xr[n][2] = xv[2];
+            xr[n][3] = xv[3];
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < TGM; ++g) {
+        const int gu = g < tga ? g : tga - 1;
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+            ColPiece pc;
+            load_piece(st, a, h ? a.q_half : 0u, h ? a.d_half : 0u, gu, col, r, pc);
+#pragma unroll
+            for (int n = 0; n < NMAX; ++n)
+                if (n < a.N)
+                    acc[g][h][n] = fmaf(dot16_x2(pc.w, xr[n][0], xr[n][1], xr[n][2], xr[n][3]), pc.d, acc[g][h][n]);
+        }
+    }
+}
+
+// TGM: the plan's row groups per CTA (1..kResTGM).
+template <int NMAX, int MODE, int TGM>
 __global__ void __launch_bounds__(kResThreads, 1)
     resident_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap td,
                     const float *__restrict__ x, const TileArgs a) {
@@ -581,16 +616,13 @@ __global__ void __launch_bounds__(kResThreads, 1)
     // units * grid < 2^31 is checked on the host, so 32-bit math is exact here
     const int u0 = (int)(((unsigned)a.units * blockIdx.x) / gridDim.x);
     const int u1 = (int)(((unsigned)a.units * (blockIdx.x + 1)) / gridDim.x);
-    const int tga = u1 - u0;  // <= kResTGM (planned on the host)
+    const int tga = u1 - u0;  // 1..TGM (planned on the host)
     if (threadIdx.x == 0) {
         mbar_init(wbar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
-    // The next kernel on the stream may start its prologue now; it reads
-    // nothing this kernel writes before its own griddepcontrol.wait.
-    pdl_launch_dependents();
     if (threadIdx.x == 0) {
         const uint64_t pw = policy_evict_first();
         const uint32_t st = smem_u32(smem);
@@ -606,8 +638,10 @@ __global__ void __launch_bounds__(kResThreads, 1)
                 }
             }
     }
-    pdl_wait();  // the activations, and the outputs, belong to the previous grid until here
-    if (MODE == kModeF32 && NMAX == 1 && tga == 1 && a.C <= kResColsPerThread * kResThreads) {
+    // the activations, and the outputs, belong to the previous grid until here;
+    // only now may the next kernel on the stream start and prefetch
+    pdl_wait_and_trigger();
+    if (MODE == kModeF32 && NMAX == 1 && TGM == 1 && a.C <= kResColsPerThread * kResThreads) {
         res_one_group(smem, a, x, u0, wbar, abort_flag, red);
         if (threadIdx.x == 0 && *abort_flag) mbar_drain(wbar, 0);
         return;
@@ -640,9 +674,9 @@ __global__ void __launch_bounds__(kResThreads, 1)
     __syncthreads();
     const bool ok = mbar_wait_warp(wbar, 0, abort_flag);
     const int r = lane & 7, j = lane >> 3;
-    float acc[kResTGM][H][NMAX];
+    float acc[TGM][H][NMAX];
 #pragma unroll
-    for (int g = 0; g < kResTGM; ++g)
+    for (int g = 0; g < TGM; ++g)
 #pragma unroll
         for (int h = 0; h < H; ++h)
 #pragma unroll
@@ -651,15 +685,12 @@ __global__ void __launch_bounds__(kResThreads, 1)
         const int nq = (a.C + 3) >> 2;
         for (int cq = warp; cq < nq; cq += kResWarps) {
             const int col = 4 * cq + j;
-            if (tga == kResTGM)
-                cols_step<NMAX, MODE, kResTGM, false>(smem, a, 0, col, a.C, r, j, tga, acc);
-            else
-                cols_step<NMAX, MODE, kResTGM, true>(smem, a, 0, col, a.C, r, j, tga, acc);
+            if (col < a.C) res_step<NMAX, MODE, TGM>(smem, a, col, r, tga, acc);
         }
     }
     // lanes r, r+8, r+16, r+24 hold partial sums of the same row
 #pragma unroll
-    for (int g = 0; g < kResTGM; ++g)
+    for (int g = 0; g < TGM; ++g)
 #pragma unroll
         for (int h = 0; h < H; ++h)
 #pragma unroll
@@ -669,12 +700,12 @@ __global__ void __launch_bounds__(kResThreads, 1)
             }
     if (j == 0) {
 #pragma unroll
-        for (int g = 0; g < kResTGM; ++g)
+        for (int g = 0; g < TGM; ++g)
 #pragma unroll
             for (int h = 0; h < H; ++h)
 #pragma unroll
                 for (int n = 0; n < NMAX; ++n)
-                    red[((((warp * kResTGM + g) * H + h) * NMAX + n) << 3) + r] = acc[g][h][n];
+                    red[((((warp * TGM + g) * H + h) * NMAX + n) << 3) + r] = acc[g][h][n];
     }
     __syncthreads();
     if (ok) {
@@ -688,7 +719,7 @@ __global__ void __launch_bounds__(kResThreads, 1)
                     float sum = 0.f;
 #pragma unroll
                     for (int w = 0; w < kResWarps; ++w)
-                        sum += red[((((w * kResTGM + g) * H + h) * NMAX + n) << 3) + rr];
+                        sum += red[((((w * TGM + g) * H + h) * NMAX + n) << 3) + rr];
                     v[h][n] = sum;
                 }
             store_unit<NMAX, MODE>(a, u0 + g, rr, v[0], v[H - 1]);
@@ -710,7 +741,7 @@ __device__ __forceinline__ void consume_groups(uint8_t *smem, uint32_t full0, ui
                                                const TileArgs &a, int u0, int u1, int n_tiles) {
     constexpr int SETS = tile_acc_sets<MODE>();
     const int cw = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane & 7, j = lane >> 3;
-    pdl_wait();  // outputs may still be read by the previous grid
+    pdl_wait_and_trigger();  // outputs may still be read by the previous grid
     int it = 0;
     for (int tl = 0; tl < n_tiles; ++tl) {
         const int ut = u0 + tl * a.TG;
@@ -842,12 +873,13 @@ __global__ void __launch_bounds__(kTileThreads, 1)
         fence_mbar_init();
     }
     __syncthreads();
-    pdl_launch_dependents();
 
     if (warp == kConsumerWarps) {
         if (lane == 0)
             tile_produce<MODE>(smem, full0, empty0, abort_flag, issued, a, u0, u1, total, &tq, &td,
                                &tq1, &td1, &tx);
+        else
+            pdl_wait_and_trigger();
     } else {
         consume_groups<NMAX, MODE>(smem, full0, empty0, red, abort_flag, a, u0, u1, n_tiles);
     }
