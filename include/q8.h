@@ -162,10 +162,12 @@ size_t q8_moe_workspace_bytes(int64_t T, int64_t E, int64_t top_k, int64_t H, in
 
 /* y[t] = sum_{s < top_k} w[t][s] * Down_e(SwiGLU(GateUp_e x[t]))  (e = idx[t][s])
  *        + Down_sh(SwiGLU(GateUp_sh x[t]))             (when a shared expert is given)
- * in two launches: one computes SwiGLU(gate_up) for every selected
- * (expert, token) pair and the shared expert, the other the down projections
- * and the weighted sum.  Each launch walks only the selected experts, and an
- * expert picked by several tokens streams its weights once.  The slot
+ * in three launches: one computes SwiGLU(gate_up) for every selected
+ * (expert, token) pair and the shared expert, one the down projection of
+ * each selected expert for its own tokens, and a small one the weighted sum.
+ * The weight launches walk only the selected experts, read only their tokens'
+ * activations, and an expert picked by several tokens streams its weights
+ * once.  The slot
  * weighting and shared expert follow the router + top-k expert +
  * shared-expert FFN block of "Add Qwen1.5-MoE Q8_0 ... - #144" (PR summary);
  * folding the per-slot launches into one grid follows the routed-expert

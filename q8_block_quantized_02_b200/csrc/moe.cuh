@@ -1,23 +1,28 @@
-// moe.cuh -- S6: grouped MoE GEMV over the routed experts, in two launches.
+// moe.cuh -- S6: grouped MoE GEMV over the routed experts, in three launches.
 //
-//   launch 1 (gate/up): for every selected expert and for the shared expert,
-//     h = SiLU(gate x) * up x for the tokens that use it.  Work units are
-//     (expert, 8-row gate group) pairs, so an expert picked by several tokens
-//     streams its weights once and serves all of them.  A routed pair's h is
+// A "segment" is one expert in use (the experts present in idx, ascending
+// id) or the shared expert (last); it serves cnt tokens.  Both weight
+// launches walk (segment, 8-row group) work items, so a selected expert's
+// weights stream once for all of its tokens and nothing else is read:
+//
+//   launch 1 (gate/up): items are (segment, gate group); each computes
+//     h = SiLU(gate x) * up x for the segment's tokens.  A routed pair's h is
 //     stored already multiplied by its routing weight, in expert-sorted pair
-//     order (pairs of one expert are consecutive rows of the workspace).
-//   launch 2 (down + sum): for every 8-row group of the output, the K stream
-//     is the concatenation of the selected experts' down rows (ascending
-//     expert id) and the shared expert's; each stage multiplies one slice of
-//     one expert by that expert's workspace rows, so y[t] is accumulated in a
-//     fixed order without atomics.
+//     order (pairs of one expert are consecutive rows of the workspace);
+//   launch 2 (down): items are (segment, output group); each multiplies the
+//     segment's down rows by the segment's h rows and writes that segment's
+//     partial output for each of its tokens, at the pair's original index
+//     t * k + s (shared expert: after them);
+//   launch 3 (sum): y[t] = the token's partials in ascending expert id, then
+//     the shared expert's: a fixed order, so results are bit-identical from
+//     run to run, and no atomics.
 //
-// Each CTA rebuilds the same expert table from idx at start (after waiting for
-// the router): experts present in idx, ascending; for each, its (token, slot)
-// pairs in token order.  The weight pipeline is the tile kernels' (producer
-// warp issuing TMA boxes into an mbarrier ring, bounded waits, drain on
-// abort); consumers use the column-owner mapping with activations read from
-// the staged box for each token of the current expert.
+// Each CTA of launches 1 and 2 rebuilds the same expert table from idx at
+// start (after waiting for the router).  The weight pipeline is the tile
+// kernels' (a producer thread issuing TMA boxes into an mbarrier ring,
+// bounded waits, drain on abort).  A stage holds CS 16-byte columns of the
+// tile's items and one TMA box per token of the segment (only the segment's
+// own activation rows); consumers use the column-owner mapping.
 #pragma once
 
 #include "tile_gemm.cuh"
@@ -36,12 +41,15 @@ struct MoeArgs {
     int T, E, k, H, I, Is;  // Is = 0: no shared expert
     const int32_t *idx;     // [T][k]
     const float *w;         // [T][k]
-    float *hbuf;            // workspace: [T*k][I] routed h (expert-sorted pairs)
+    float *hbuf;            // workspace: [T*k][I] routed h (expert-sorted pair rows)
     float *hsh;             // workspace: [T][Is] shared h
+    float *part;            // workspace: [T*k + T][H] partial outputs of launch 2
     float *y;               // [T][H]
-    int units_out;          // launch 2: H / 8
     int TG, CS, stages;
-    uint32_t q_box, d_box, x_box, q_half, d_off, d_half, x_off, stage_bytes;
+    uint32_t q_box;         // bytes of one item's q box (CS * 128)
+    uint32_t d_box;         // bytes of one item's scale box (CS * 8)
+    uint32_t x_row;         // bytes of one token's activation box (CS * 64)
+    uint32_t q_half, d_off, d_half, x_off, stage_bytes;
 };
 
 struct MoeTable {
@@ -50,16 +58,17 @@ struct MoeTable {
     int seg_expert[kMoeMaxSeg];        // expert id, -1 for the shared expert
     int seg_row0[kMoeMaxSeg];          // first pair row (routed)
     int seg_cnt[kMoeMaxSeg];           // tokens using it
-    int seg_unit0[kMoeMaxSeg + 1];     // launch 1: first flattened unit
-    int seg_kstep0[kMoeMaxSeg + 1];    // launch 2: first stage of the segment in a tile
+    int seg_unit0[kMoeMaxSeg + 1];     // first work item (flattened, for this launch)
     short pair_tok[kMoeMaxPairs];      // pair row -> token
     short pair_slot[kMoeMaxPairs];     // pair row -> slot
-    signed char box_row[kMoeMaxSeg][kMoeMaxT];  // launch 2: token -> row of the x box, or -1
     int counts[kMoeMaxE];
 };
 
 // Build the table with all threads of the CTA (idx must be readable).
-__device__ __forceinline__ void moe_build_table(MoeTable &tb, const MoeArgs &a, int stage_kind) {
+// `items_routed` / `items_shared`: work items of one routed / the shared
+// segment in this launch.
+__device__ __forceinline__ void moe_build_table(MoeTable &tb, const MoeArgs &a, int items_routed,
+                                                int items_shared) {
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int P = a.T * a.k;
     for (int e = tid; e < kMoeMaxE; e += nthr) tb.counts[e] = 0;
@@ -124,32 +133,13 @@ __device__ __forceinline__ void moe_build_table(MoeTable &tb, const MoeArgs &a, 
         tb.pair_tok[row] = (short)(p / a.k);
         tb.pair_slot[row] = (short)(p % a.k);
     }
-    __syncthreads();
     if (tid == 0) {
-        // launch 1 unit offsets; launch 2 stage offsets (per tile)
-        int u = 0, ks = 0;
-        const int c_routed = a.I / 16, c_shared = a.Is / 16;
+        int u = 0;
         for (int s = 0; s < tb.n_seg; ++s) {
             tb.seg_unit0[s] = u;
-            tb.seg_kstep0[s] = ks;
-            const bool shared = tb.seg_expert[s] < 0;
-            u += (shared ? a.Is : a.I) / kGroupRows;
-            ks += ((shared ? c_shared : c_routed) + a.CS - 1) / a.CS;
+            u += tb.seg_expert[s] < 0 ? items_shared : items_routed;
         }
         tb.seg_unit0[tb.n_seg] = u;
-        tb.seg_kstep0[tb.n_seg] = ks;
-    }
-    if (stage_kind == 2) {
-        for (int i = tid; i < kMoeMaxSeg * kMoeMaxT; i += nthr) (&tb.box_row[0][0])[i] = -1;
-        __syncthreads();
-        for (int s = tid; s < tb.n_seg; s += nthr) {
-            if (tb.seg_expert[s] < 0) {
-                for (int t = 0; t < a.T; ++t) tb.box_row[s][t] = (signed char)t;
-            } else {
-                for (int i = 0; i < tb.seg_cnt[s]; ++i)
-                    tb.box_row[s][tb.pair_tok[tb.seg_row0[s] + i]] = (signed char)i;
-            }
-        }
     }
     __syncthreads();
 }
@@ -162,7 +152,7 @@ __device__ __forceinline__ void moe_load_piece(const uint8_t *st, const MoeArgs 
     dequant16_x2(q, p.w);
 }
 
-// index of the segment holding flattened launch-1 unit u
+// index of the segment holding flattened work item u
 __device__ __forceinline__ int moe_seg_of_unit(const MoeTable &tb, int u) {
     int lo = 0, hi = tb.n_seg - 1;
     while (lo < hi) {
@@ -172,27 +162,136 @@ __device__ __forceinline__ int moe_seg_of_unit(const MoeTable &tb, int u) {
     return lo;
 }
 
-__device__ __forceinline__ int moe_seg_of_kstep(const MoeTable &tb, int ks) {
-    int lo = 0, hi = tb.n_seg - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (tb.seg_kstep0[mid] <= ks) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
-
-// Tiles of launch 1: runs of <= TG consecutive units of one segment inside the
-// CTA's range.  Walk them with this cursor.
+// Tiles: runs of <= TG consecutive items of one segment inside the CTA's
+// range.  Walk them with this cursor.
 struct MoeTile {
-    int seg, ut, tga;  // segment, first unit (flattened), units
+    int seg, ut, tga;  // segment, first item (flattened), items
 };
 
-__device__ __forceinline__ MoeTile moe_tile1(const MoeTable &tb, const MoeArgs &a, int u, int u1) {
+__device__ __forceinline__ MoeTile moe_tile(const MoeTable &tb, const MoeArgs &a, int u, int u1) {
     MoeTile t;
     t.seg = moe_seg_of_unit(tb, u);
     t.ut = u;
     t.tga = min(min(a.TG, u1 - u), tb.seg_unit0[t.seg + 1] - u);
     return t;
+}
+
+// K of a segment in 16-byte columns: launch 1 reads x (H wide) for every
+// segment; launch 2 reads the segment's h (I wide, Is for the shared expert).
+template <int STAGE>
+__device__ __forceinline__ int moe_seg_cols(const MoeArgs &a, bool shared) {
+    return STAGE == 1 ? a.H / 16 : (shared ? a.Is : a.I) / 16;
+}
+
+// The stages of one tile for a consumer warp: NX >= cnt token entries (a
+// compile-time bound, so the per-token chains unroll), TGM items with no
+// per-item branch (a tile with fewer items recomputes its last one; those
+// sums are never stored).  Leaves the warp's per-row partials in `red`.
+template <int STAGE, int NX, int TGM, int NMAX>
+__device__ __forceinline__ void moe_tile_compute(const uint8_t *smem, const MoeArgs &a, uint32_t full0,
+                                                 uint32_t empty0, volatile int *abort_flag, int &it, int ks_n,
+                                                 int cols_seg, int tga, int cnt, float *red) {
+    constexpr int H = STAGE == 1 ? 2 : 1;
+    const int cw = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane & 7, j = lane >> 3;
+    float acc[TGM][H][NX];
+#pragma unroll
+    for (int g = 0; g < TGM; ++g)
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+#pragma unroll
+            for (int n = 0; n < NX; ++n) acc[g][h][n] = 0.f;
+    for (int ks = 0; ks < ks_n; ++ks, ++it) {
+        const int slot = it % a.stages;
+        if (mbar_wait_warp(full0 + 8 * slot, (it / a.stages) & 1, abort_flag)) {
+            const uint8_t *st = smem + (size_t)slot * a.stage_bytes;
+            const int cols = min(a.CS, cols_seg - ks * a.CS);
+            const int nq = (cols + 3) >> 2;
+            for (int cq = cw; cq < nq; cq += kMoeWarps) {
+                const int col = 4 * cq + j;
+                if (col >= cols) continue;
+                // token entries past cnt read row cnt - 1 again (unstored); up to
+                // four tokens' activations stay in registers for all items
+                constexpr int XR = NX <= 4 ? NX : 1;
+                ulonglong2 xr[XR][4];
+                if (NX <= 4) {
+#pragma unroll
+                    for (int n = 0; n < XR; ++n) {
+                        const int nn = n < cnt ? n : cnt - 1;
+                        const ulonglong2 *xv =
+                            reinterpret_cast<const ulonglong2 *>(st + a.x_off + nn * a.x_row + col * 64);
+                        xr[n][0] = xv[0];
+                        xr[n][1] = xv[1];
+                        xr[n][2] = xv[2];
+                        xr[n][3] = xv[3];
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < TGM; ++g) {
+                    const int gu = g < tga ? g : tga - 1;
+#pragma unroll
+                    for (int h = 0; h < H; ++h) {
+                        ColPiece pc;
+                        moe_load_piece(st, a, h ? a.q_half : 0u, h ? a.d_half : 0u, gu, col, r, pc);
+#pragma unroll
+                        for (int n = 0; n < NX; ++n) {
+                            if (NX <= 4) {
+                                acc[g][h][n] = fmaf(dot16_x2(pc.w, xr[n % XR][0], xr[n % XR][1], xr[n % XR][2],
+                                                             xr[n % XR][3]),
+                                                    pc.d, acc[g][h][n]);
+                            } else {
+                                const int nn = n < cnt ? n : cnt - 1;
+                                const ulonglong2 *xv =
+                                    reinterpret_cast<const ulonglong2 *>(st + a.x_off + nn * a.x_row + col * 64);
+                                acc[g][h][n] = fmaf(dot16_x2(pc.w, xv[0], xv[1], xv[2], xv[3]), pc.d, acc[g][h][n]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * slot);
+    }
+#pragma unroll
+    for (int g = 0; g < TGM; ++g)
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+#pragma unroll
+            for (int n = 0; n < NX; ++n) {
+                acc[g][h][n] += __shfl_xor_sync(0xffffffffu, acc[g][h][n], 8);
+                acc[g][h][n] += __shfl_xor_sync(0xffffffffu, acc[g][h][n], 16);
+            }
+    if (j == 0) {
+#pragma unroll
+        for (int g = 0; g < TGM; ++g)
+#pragma unroll
+            for (int h = 0; h < H; ++h)
+#pragma unroll
+                for (int n = 0; n < NX; ++n)
+                    red[((((cw * TGM + g) * H + h) * NMAX + n) << 3) + r] = acc[g][h][n];
+    }
+}
+
+// First work item of CTA c of `grid`: the first item starting at or after
+// work position W * c / grid, where an item's work is its segment's stage
+// count and W the total.  Monotone in c, 0 at c = 0 and U at c = grid, so the
+// CTAs' ranges partition the items.
+template <int STAGE>
+__device__ __forceinline__ int moe_work_split(const MoeTable &tb, const MoeArgs &a, int c, int grid) {
+    long long W = 0;
+    for (int s = 0; s < tb.n_seg; ++s) {
+        const int ks = (moe_seg_cols<STAGE>(a, tb.seg_expert[s] < 0) + a.CS - 1) / a.CS;
+        W += (long long)(tb.seg_unit0[s + 1] - tb.seg_unit0[s]) * ks;
+    }
+    const long long P = W * c / grid;
+    long long w0 = 0;
+    for (int s = 0; s < tb.n_seg; ++s) {
+        const int ks = (moe_seg_cols<STAGE>(a, tb.seg_expert[s] < 0) + a.CS - 1) / a.CS;
+        const long long ws = (long long)(tb.seg_unit0[s + 1] - tb.seg_unit0[s]) * ks;
+        if (P < w0 + ws) return tb.seg_unit0[s] + (int)((P - w0 + ks - 1) / ks);
+        w0 += ws;
+    }
+    return tb.seg_unit0[tb.n_seg];
 }
 
 template <int STAGE, int NMAX, int TGM>
@@ -213,23 +312,19 @@ __global__ void __launch_bounds__(kMoeThreads, 1)
     volatile int *issued = abort_flag + 1;
 
     pdl_wait_and_trigger();  // idx, w (router) and the activations come from earlier kernels
-    moe_build_table(tb, a, STAGE);
+    moe_build_table(tb, a, (STAGE == 1 ? a.I : a.H) / kGroupRows, (STAGE == 1 ? a.Is : a.H) / kGroupRows);
 
-    // this CTA's range of units
-    const int U = STAGE == 1 ? tb.seg_unit0[tb.n_seg] : a.units_out;
-    const int u0 = (int)(((long long)U * blockIdx.x) / gridDim.x);
-    const int u1 = (int)(((long long)U * (blockIdx.x + 1)) / gridDim.x);
-    const int ksteps2 = tb.seg_kstep0[tb.n_seg];  // launch 2: stages per tile
-    const int ksteps1 = (a.H / 16 + a.CS - 1) / a.CS;
-    const int ksteps = STAGE == 1 ? ksteps1 : ksteps2;
-    // count the tiles and stages of this CTA
-    int n_tiles = 0;
+    // this CTA's range of work items, balanced by work (an item's stages:
+    // the shared expert's down items are longer), then its tiles and stages
+    const int u0 = moe_work_split<STAGE>(tb, a, blockIdx.x, gridDim.x);
+    const int u1 = moe_work_split<STAGE>(tb, a, blockIdx.x + 1, gridDim.x);
+    int n_tiles = 0, total = 0;
     for (int u = u0; u < u1;) {
-        const int step = STAGE == 1 ? moe_tile1(tb, a, u, u1).tga : min(a.TG, u1 - u);
-        u += step;
+        const MoeTile t = moe_tile(tb, a, u, u1);
+        u += t.tga;
         ++n_tiles;
+        total += (moe_seg_cols<STAGE>(a, tb.seg_expert[t.seg] < 0) + a.CS - 1) / a.CS;
     }
-    const int total = n_tiles * ksteps;
     const int used_stages = total < a.stages ? total : a.stages;
     if (threadIdx.x == 0) {
         for (int s = 0; s < used_stages; ++s) {
@@ -248,40 +343,36 @@ __global__ void __launch_bounds__(kMoeThreads, 1)
             const uint64_t pw = policy_evict_first(), px = policy_evict_last();
             int it = 0, u = u0;
             for (int tl = 0; tl < n_tiles; ++tl) {
-                MoeTile t;
-                if (STAGE == 1) {
-                    t = moe_tile1(tb, a, u, u1);
-                } else {
-                    t.seg = 0;
-                    t.ut = u;
-                    t.tga = min(a.TG, u1 - u);
-                }
+                const MoeTile t = moe_tile(tb, a, u, u1);
                 u += t.tga;
-                for (int ks = 0; ks < ksteps; ++ks, ++it) {
+                const bool shared = tb.seg_expert[t.seg] < 0;
+                const int ks_n = (moe_seg_cols<STAGE>(a, shared) + a.CS - 1) / a.CS;
+                const int cnt = tb.seg_cnt[t.seg], row0 = tb.seg_row0[t.seg];
+                const int in_seg = t.ut - tb.seg_unit0[t.seg];
+                // packed group of the tile's first item, and the gate -> up distance
+                int g0, up;
+                if (STAGE == 1) {
+                    const int gates = (shared ? a.Is : a.I) / kGroupRows;
+                    g0 = (shared ? 0 : tb.seg_expert[t.seg] * 2 * gates) + in_seg;
+                    up = gates;
+                } else {
+                    g0 = (shared ? 0 : tb.seg_expert[t.seg] * (a.H / kGroupRows)) + in_seg;
+                    up = 0;
+                }
+                const CUtensorMap *mq = shared ? &tq_s : &tq_r;
+                const CUtensorMap *md = shared ? &td_s : &td_r;
+                const CUtensorMap *mx = (STAGE == 2 && shared) ? &tx_s : &tx_r;
+                for (int ks = 0; ks < ks_n; ++ks, ++it) {
                     const int slot = it % a.stages;
                     if (it >= a.stages && !mbar_wait(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag)) {
                         *issued = it;
                         goto producer_done;
                     }
                     {
-                        const int seg = STAGE == 1 ? t.seg : moe_seg_of_kstep(tb, ks);
-                        const bool shared = tb.seg_expert[seg] < 0;
-                        const int c0 = (STAGE == 1 ? ks : ks - tb.seg_kstep0[seg]) * a.CS;
+                        const int c0 = ks * a.CS;
                         const uint32_t st = smem_u32(smem + (size_t)slot * a.stage_bytes);
                         const uint32_t full = full0 + 8 * slot;
-                        const CUtensorMap *mq = shared ? &tq_s : &tq_r;
-                        const CUtensorMap *md = shared ? &td_s : &td_r;
-                        mbar_arrive_expect_tx(full, H * t.tga * (a.q_box + a.d_box) + a.x_box);
-                        int g0, up;
-                        if (STAGE == 1) {
-                            const int in_seg = t.ut - tb.seg_unit0[seg];
-                            const int gates = (shared ? a.Is : a.I) / kGroupRows;
-                            g0 = (shared ? 0 : tb.seg_expert[seg] * 2 * gates) + in_seg;
-                            up = gates;
-                        } else {
-                            g0 = (shared ? 0 : tb.seg_expert[seg] * (a.H / kGroupRows)) + t.ut;
-                            up = 0;
-                        }
+                        mbar_arrive_expect_tx(full, H * t.tga * (a.q_box + a.d_box) + cnt * a.x_row);
                         for (int g = 0; g < t.tga; ++g)
 #pragma unroll
                             for (int h = 0; h < H; ++h) {
@@ -289,12 +380,11 @@ __global__ void __launch_bounds__(kMoeThreads, 1)
                                 tma_load_3d(st + a.d_off + (h ? a.d_half : 0u) + g * a.d_box, md, full, 0, c0 >> 1,
                                             g0 + g + h * up, pw);
                             }
-                        if (STAGE == 1)
-                            tma_load_3d(st + a.x_off, &tx_r, full, 0, c0, 0, px);
-                        else if (shared)
-                            tma_load_3d(st + a.x_off, &tx_s, full, 0, c0, 0, px);
-                        else
-                            tma_load_3d(st + a.x_off, &tx_r, full, 0, c0, tb.seg_row0[seg], px);
+                        // the segment's own activation rows, one box each
+                        for (int n = 0; n < cnt; ++n) {
+                            const int row = shared ? n : (STAGE == 1 ? (int)tb.pair_tok[row0 + n] : row0 + n);
+                            tma_load_3d(st + a.x_off + n * a.x_row, mx, full, 0, c0, row, px);
+                        }
                     }
                 }
             }
@@ -303,94 +393,33 @@ __global__ void __launch_bounds__(kMoeThreads, 1)
         }
     } else {
         // ------------------------------ consumers -----------------------------
-        const int cw = warp, r = lane & 7, j = lane >> 3;
         int it = 0, u = u0;
         for (int tl = 0; tl < n_tiles; ++tl) {
-            MoeTile t;
-            if (STAGE == 1) {
-                t = moe_tile1(tb, a, u, u1);
-            } else {
-                t.seg = 0;
-                t.ut = u;
-                t.tga = min(a.TG, u1 - u);
-            }
+            const MoeTile t = moe_tile(tb, a, u, u1);
             u += t.tga;
-            float acc[TGM][H][NMAX];
-#pragma unroll
-            for (int g = 0; g < TGM; ++g)
-#pragma unroll
-                for (int h = 0; h < H; ++h)
-#pragma unroll
-                    for (int n = 0; n < NMAX; ++n) acc[g][h][n] = 0.f;
-            for (int ks = 0; ks < ksteps; ++ks, ++it) {
-                const int slot = it % a.stages;
-                if (mbar_wait(full0 + 8 * slot, (it / a.stages) & 1, abort_flag)) {
-                    const uint8_t *st = smem + (size_t)slot * a.stage_bytes;
-                    const int seg = STAGE == 1 ? t.seg : moe_seg_of_kstep(tb, ks);
-                    const bool shared = tb.seg_expert[seg] < 0;
-                    const int cseg = (shared ? a.Is : (STAGE == 1 ? a.H : a.I)) / 16;
-                    const int c_here = (STAGE == 1 ? a.H / 16 : cseg);
-                    const int c0 = (STAGE == 1 ? ks : ks - tb.seg_kstep0[seg]) * a.CS;
-                    const int cols = min(a.CS, c_here - c0);
-                    const int nq = (cols + 3) >> 2;
-                    const int cnt = tb.seg_cnt[seg];
-                    for (int cq = cw; cq < nq; cq += kMoeWarps) {
-                        const int col = 4 * cq + j;
-                        if (col >= cols) continue;
-#pragma unroll
-                        for (int g = 0; g < TGM; ++g) {
-                            if (g < t.tga) {
-#pragma unroll
-                                for (int h = 0; h < H; ++h) {
-                                    ColPiece pc;
-                                    moe_load_piece(st, a, h ? a.q_half : 0u, h ? a.d_half : 0u, g, col, r, pc);
-#pragma unroll
-                                    for (int n = 0; n < NMAX; ++n) {
-                                        // launch 1: entry n of the segment's token list;
-                                        // launch 2: token n, read from its box row
-                                        int row;
-                                        if (STAGE == 1)
-                                            row = n < cnt ? (shared ? n : tb.pair_tok[tb.seg_row0[seg] + n]) : -1;
-                                        else
-                                            row = n < a.T ? tb.box_row[seg][n] : -1;
-                                        if (row >= 0) {
-                                            const ulonglong2 *xv = reinterpret_cast<const ulonglong2 *>(
-                                                st + a.x_off + (row * a.CS + col) * 64);
-                                            acc[g][h][n] = fmaf(dot16_x2(pc.w, xv[0], xv[1], xv[2], xv[3]), pc.d,
-                                                                acc[g][h][n]);
-                                        }
-                                    }
-                                }
-                            }
-                        }
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty0 + 8 * slot);
-            }
-#pragma unroll
-            for (int g = 0; g < TGM; ++g)
-#pragma unroll
-                for (int h = 0; h < H; ++h)
-#pragma unroll
-                    for (int n = 0; n < NMAX; ++n) {
-                        acc[g][h][n] += __shfl_xor_sync(0xffffffffu, acc[g][h][n], 8);
-                        acc[g][h][n] += __shfl_xor_sync(0xffffffffu, acc[g][h][n], 16);
-                    }
-            if (j == 0) {
-#pragma unroll
-                for (int g = 0; g < TGM; ++g)
-#pragma unroll
-                    for (int h = 0; h < H; ++h)
-#pragma unroll
-                        for (int n = 0; n < NMAX; ++n)
-                            red[((((cw * TGM + g) * H + h) * NMAX + n) << 3) + r] = acc[g][h][n];
-            }
+            const bool shared = tb.seg_expert[t.seg] < 0;
+            const int cols_seg = moe_seg_cols<STAGE>(a, shared);
+            const int ks_n = (cols_seg + a.CS - 1) / a.CS;
+            const int cnt = tb.seg_cnt[t.seg];
+            // the segment's token count, rounded up to a power of two <= NMAX
+            if (NMAX == 1 || cnt <= 1)
+                moe_tile_compute<STAGE, 1, TGM, NMAX>(smem, a, full0, empty0, abort_flag, it, ks_n, cols_seg, t.tga, cnt, red);
+            else if (NMAX == 2 || cnt <= 2)
+                moe_tile_compute<STAGE, (NMAX < 2 ? NMAX : 2), TGM, NMAX>(smem, a, full0, empty0, abort_flag, it, ks_n,
+                                                                          cols_seg, t.tga, cnt, red);
+            else if (NMAX == 4 || cnt <= 4)
+                moe_tile_compute<STAGE, (NMAX < 4 ? NMAX : 4), TGM, NMAX>(smem, a, full0, empty0, abort_flag, it, ks_n,
+                                                                          cols_seg, t.tga, cnt, red);
+            else if (NMAX == 8 || cnt <= 8)
+                moe_tile_compute<STAGE, (NMAX < 8 ? NMAX : 8), TGM, NMAX>(smem, a, full0, empty0, abort_flag, it, ks_n,
+                                                                          cols_seg, t.tga, cnt, red);
+            else
+                moe_tile_compute<STAGE, NMAX, TGM, NMAX>(smem, a, full0, empty0, abort_flag, it, ks_n, cols_seg,
+                                                         t.tga, cnt, red);
             named_barrier(1, kMoeWarps * 32);
-            // outputs: (unit g, row r, entry n), warps' partials added in warp order
-            const int seg = t.seg;
-            const bool shared = STAGE == 1 && tb.seg_expert[seg] < 0;
-            const int cnt = STAGE == 1 ? tb.seg_cnt[seg] : a.T;
+            // outputs: (item g, row rr, token entry n), warps' partials added in warp order
+            const int in_seg = t.ut - tb.seg_unit0[t.seg];
+            const int row0 = tb.seg_row0[t.seg];
             for (int o = threadIdx.x; o < t.tga * 8 * NMAX; o += kMoeWarps * 32) {
                 const int n = o % NMAX, rr = (o / NMAX) & 7, g = o / (NMAX * 8);
                 if (n >= cnt) continue;
@@ -402,17 +431,18 @@ __global__ void __launch_bounds__(kMoeThreads, 1)
                     for (int w = 0; w < kMoeWarps; ++w) s += red[((((w * TGM + g) * H + h) * NMAX + n) << 3) + rr];
                     v[h] = s;
                 }
+                const int row = (in_seg + g) * kGroupRows + rr;  // row of h (launch 1) or of y (launch 2)
                 if (STAGE == 1) {
                     const float hval = silu_mul(v[0], v[H - 1]);
-                    const int row = (t.ut - tb.seg_unit0[seg] + g) * kGroupRows + rr;
                     if (shared) {
                         a.hsh[(size_t)n * a.Is + row] = hval;
                     } else {
-                        const int pr = tb.seg_row0[seg] + n;
+                        const int pr = row0 + n;
                         a.hbuf[(size_t)pr * a.I + row] = hval * a.w[tb.pair_tok[pr] * a.k + tb.pair_slot[pr]];
                     }
                 } else {
-                    a.y[(size_t)n * a.H + (t.ut + g) * kGroupRows + rr] = v[0];
+                    const int dst = shared ? a.T * a.k + n : tb.pair_tok[row0 + n] * a.k + tb.pair_slot[row0 + n];
+                    a.part[(size_t)dst * a.H + row] = v[0];
                 }
             }
             named_barrier(1, kMoeWarps * 32);
@@ -423,6 +453,37 @@ __global__ void __launch_bounds__(kMoeThreads, 1)
         const int n_issued = *issued;
         for (int it = n_issued > a.stages ? n_issued - a.stages : 0; it < n_issued; ++it)
             mbar_drain(full0 + 8 * (it % a.stages), (it / a.stages) & 1);
+    }
+}
+
+// Launch 3: y[t][h] = the token's routed partials in ascending expert id (a
+// repeated pick of one expert in slot order), then the shared expert's.  An
+// out-of-range pick contributes nothing.
+__global__ void moe_sum_kernel(const int32_t *__restrict__ idx, const float *__restrict__ part,
+                               float *__restrict__ y, int T, int E, int k, int H, int has_shared) {
+    pdl_wait_and_trigger();
+    const int total = T * H;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+        const int t = i / H, h = i - t * H;
+        float s = 0.f;
+        int last = -1;  // key e * k + slot of the pick added last
+        for (int r = 0; r < k; ++r) {
+            int best = -1, best_key = 0x7fffffff;
+            for (int q = 0; q < k; ++q) {
+                const int e = idx[t * k + q];
+                if (e < 0 || e >= E) continue;
+                const int key = e * k + q;
+                if (key > last && key < best_key) {
+                    best_key = key;
+                    best = q;
+                }
+            }
+            if (best < 0) break;
+            s += part[(size_t)(t * k + best) * H + h];
+            last = best_key;
+        }
+        if (has_shared) s += part[(size_t)(T * k + t) * H + h];
+        y[i] = s;
     }
 }
 

@@ -417,17 +417,21 @@ static q8_status run_mma(const void *W, const int8_t *xq, const uint16_t *xd, fl
 using MoeKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
                            CUtensorMap, MoeArgs);
 
-template <int STAGE, int NMAX>
-static MoeKernel moe_kernel_ptr() {
-    constexpr int TGM = STAGE == 1 ? (32 / NMAX < 1 ? 1 : 32 / NMAX > 8 ? 8 : 32 / NMAX)
-                                   : (64 / NMAX > 8 ? 8 : 64 / NMAX);
-    return &moe_kernel<STAGE, NMAX, TGM>;
+// Items per tile: as many as ~32 KB of weights hold at 32 columns a stage
+// (3 gate|up items, 7 down items), and at most 32 fp32 accumulators per lane
+// (items x halves x tokens).  The kernel computes exactly this many, so a
+// full tile wastes nothing.
+__host__ __device__ constexpr int moe_tgm_c(int stage, int nmax) {
+    return stage == 1 ? (16 / nmax < 1 ? 1 : 16 / nmax < 3 ? 16 / nmax : 3)
+                      : (32 / nmax < 7 ? 32 / nmax : 7);
 }
 
-static int moe_tgm(int stage, int nmax) {
-    const int v = (stage == 1 ? 32 : 64) / nmax;
-    return v < 1 ? 1 : v > 8 ? 8 : v;
+template <int STAGE, int NMAX>
+static MoeKernel moe_kernel_ptr() {
+    return &moe_kernel<STAGE, NMAX, moe_tgm_c(STAGE, NMAX)>;
 }
+
+static int moe_tgm(int stage, int nmax) { return moe_tgm_c(stage, nmax); }
 
 static MoeKernel moe_kernel_for(int stage, int nmax) {
     switch (nmax) {
@@ -460,38 +464,47 @@ struct MoePlan {
     size_t smem;
 };
 
-// Stage shape for a MoE launch: TG units of `halves` weight boxes of CS
-// columns (~32 KB) plus the activation box of T rows (<= 16 KB).
+// Stage shape for a MoE weight launch: TG items of `halves` weight boxes of
+// CS columns (about 32 KB of weights) and one activation box per token of the
+// segment (T at most).  These launches cannot prefetch weights before their
+// dependency wait (the router picks them), so the ring takes most of the
+// SM's shared memory to keep several stages in flight.
 static MoePlan plan_moe(int stage, int64_t T, int64_t c_min, int nmax, int64_t units_bound, int sms) {
     MoePlan p;
     MoeArgs &a = p.a;
     a = MoeArgs{};
     const int halves = stage == 1 ? 2 : 1;
-    const int tg = moe_tgm(stage, nmax);
-    int64_t cs = (32 * 1024) / ((int64_t)tg * halves * 136) / 16 * 16;
-    const int64_t cs_x = (16 * 1024) / (T * 64) / 16 * 16;
-    cs = std::min<int64_t>(cs, cs_x);
-    cs = std::min<int64_t>(cs, round_up(c_min, 16));
-    if (cs < 16) cs = 16;
+    p.grid = (int)std::max<int64_t>(1, std::min<int64_t>(sms, units_bound));
+    const int64_t upc = ceil_div(units_bound, p.grid);
+    // 32 columns (8 quads: one per consumer warp) unless K or the activation
+    // boxes are smaller; then as many items as keep ~32 KB of weights a stage
+    int64_t cs = std::min<int64_t>(32, round_up(c_min, 16));
+    const int64_t cs_x = (32 * 1024) / (T * 64) / 16 * 16;
+    cs = std::max<int64_t>(16, std::min<int64_t>(cs, cs_x));
+    const int64_t tg_bytes = std::max<int64_t>(1, (32 * 1024) / (halves * cs * 136));
+    const int tg = (int)std::min<int64_t>(std::min<int64_t>(moe_tgm(stage, nmax), upc), tg_bytes);
     a.TG = tg;
     a.CS = (int)cs;
     a.q_box = (uint32_t)(cs * kColBytes);
     a.d_box = (uint32_t)(cs * 8);
-    a.x_box = (uint32_t)(T * cs * 64);
+    a.x_row = (uint32_t)(cs * 64);
     a.q_half = (uint32_t)tg * a.q_box;
     a.d_off = halves * a.q_half;
     a.d_half = (uint32_t)tg * a.d_box;
     a.x_off = a.d_off + halves * a.d_half;
-    a.stage_bytes = (uint32_t)round_up(a.x_off + a.x_box, 128);
-    const size_t fixed = sizeof(MoeTable) + (size_t)kMoeWarps * tg * halves * nmax * 8 * 4 + 16;
-    int64_t stages = (int64_t)(104 * 1024 - fixed) / a.stage_bytes;
-    a.stages = (int)(stages < 2 ? 2 : stages > 6 ? 6 : stages);
-    p.grid = (int)std::min<int64_t>(sms, units_bound);
+    a.stage_bytes = (uint32_t)round_up(a.x_off + T * a.x_row, 128);
+    const size_t fixed =
+        sizeof(MoeTable) + (size_t)kMoeWarps * moe_tgm(stage, nmax) * halves * nmax * 8 * 4 + 16;
+    const int64_t stages = (int64_t)(190 * 1024 - fixed) / a.stage_bytes;
+    a.stages = (int)(stages < 2 ? 2 : stages > 8 ? 8 : stages);
     p.smem = (size_t)a.stages * a.stage_bytes + 16 * a.stages + fixed;
     return p;
 }
 
 static size_t moe_hbuf_bytes(int64_t T, int64_t k, int64_t I) { return (size_t)round_up(T * k * I * 4, 256); }
+static size_t moe_hsh_bytes(int64_t T, int64_t Is) { return (size_t)round_up(T * Is * 4, 256); }
+// launch 2's partial outputs: one row per (token, slot) pair, then one per token
+static size_t moe_part_bytes(int64_t T, int64_t k, int64_t H) { return (size_t)round_up((T * k + T) * H * 4, 256); }
 
 // ---------------------------------------------------------------------------
 // scratch for q8_moe_gemv_noalloc: a fixed array in the library's own device
@@ -679,7 +692,7 @@ q8_status q8_moe_route(const float *logits, int64_t T, int64_t E, int64_t top_k,
 size_t q8_moe_workspace_bytes(int64_t T, int64_t E, int64_t top_k, int64_t H, int64_t I,
                               int64_t I_shared) {
     if (T <= 0 || E <= 0 || top_k <= 0 || H <= 0 || I <= 0 || I_shared < 0) return 0;
-    return moe_hbuf_bytes(T, top_k, I) + (size_t)round_up(T * I_shared * 4, 256);
+    return moe_hbuf_bytes(T, top_k, I) + moe_hsh_bytes(T, I_shared) + moe_part_bytes(T, top_k, H);
 }
 
 q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
@@ -714,6 +727,8 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
     cudaStream_t s = (cudaStream_t)stream;
     float *hbuf = static_cast<float *>(workspace);
     float *hsh = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + moe_hbuf_bytes(T, top_k, I));
+    float *part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + moe_hbuf_bytes(T, top_k, I) +
+                                            moe_hsh_bytes(T, I_shared));
     const int nb = nmax_for(T);
     const int64_t Ish = has_shared ? I_shared : 0;
 
@@ -723,8 +738,7 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
         MoePlan p = plan_moe(1, T, H / 16, nb, units_bound, dev->sms);
         MoeArgs &a = p.a;
         a.T = (int)T; a.E = (int)E; a.k = (int)top_k; a.H = (int)H; a.I = (int)I; a.Is = (int)Ish;
-        a.idx = idx; a.w = w; a.hbuf = hbuf; a.hsh = hsh; a.y = y;
-        a.units_out = (int)(H / 8);
+        a.idx = idx; a.w = w; a.hbuf = hbuf; a.hsh = hsh; a.part = part; a.y = y;
         if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
         const uint64_t gs = (uint64_t)kGroupBytesPerBlock * (H / 32);
         CUtensorMap tq_r, td_r, tq_s, td_s, tx;
@@ -741,18 +755,18 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
                              static_cast<const uint8_t *>(sgu) + 256 * (H / 32), 8, H / 32, sg, 16, gs, 8,
                              a.CS / 2, 1, true));
         Q8_CHECK(make_map_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, H / 16, T, 64, (uint64_t)H * 4, 16,
-                             a.CS, (uint32_t)T, false));
+                             a.CS, 1, false));
         Q8_CHECK(launch_pdl(moe_kernel_for(1, nb), dim3(p.grid), dim3(kMoeThreads), p.smem, s,
                             "q8_moe_gemv gate_up launch", tq_r, td_r, tq_s, td_s, tx, tx, a));
     }
-    // ---- launch 2: down projections, summed per output row group
+    // ---- launch 2: down projection of each selected expert for its tokens
     {
         const int64_t c_min = has_shared ? std::min<int64_t>(I, Ish) / 16 : I / 16;
-        MoePlan p = plan_moe(2, T, c_min, nb, H / 8, dev->sms);
+        const int64_t units_bound = (std::min<int64_t>(T * top_k, E) + (has_shared ? 1 : 0)) * (H / 8);
+        MoePlan p = plan_moe(2, T, c_min, nb, units_bound, dev->sms);
         MoeArgs &a = p.a;
         a.T = (int)T; a.E = (int)E; a.k = (int)top_k; a.H = (int)H; a.I = (int)I; a.Is = (int)Ish;
-        a.idx = idx; a.w = w; a.hbuf = hbuf; a.hsh = hsh; a.y = y;
-        a.units_out = (int)(H / 8);
+        a.idx = idx; a.w = w; a.hbuf = hbuf; a.hsh = hsh; a.part = part; a.y = y;
         if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
         const uint64_t gs_r = (uint64_t)kGroupBytesPerBlock * (I / 32);
         CUtensorMap tq_r, td_r, tq_s, td_s, tx_r, tx_s;
@@ -762,7 +776,7 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
                              static_cast<const uint8_t *>(down_experts) + 256 * (I / 32), 8, I / 32,
                              E * (H / 8), 16, gs_r, 8, a.CS / 2, 1, true));
         Q8_CHECK(make_map_3d(&tx_r, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, hbuf, 16, I / 16, T * top_k, 64,
-                             (uint64_t)I * 4, 16, a.CS, (uint32_t)T, false));
+                             (uint64_t)I * 4, 16, a.CS, 1, false));
         if (has_shared) {
             const uint64_t gs_s = (uint64_t)kGroupBytesPerBlock * (Ish / 32);
             Q8_CHECK(make_map_3d(&tq_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, shared_down, kColBytes, Ish / 16, H / 8,
@@ -771,7 +785,7 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
                                  static_cast<const uint8_t *>(shared_down) + 256 * (Ish / 32), 8, Ish / 32,
                                  H / 8, 16, gs_s, 8, a.CS / 2, 1, true));
             Q8_CHECK(make_map_3d(&tx_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, hsh, 16, Ish / 16, T, 64,
-                                 (uint64_t)Ish * 4, 16, a.CS, (uint32_t)T, false));
+                                 (uint64_t)Ish * 4, 16, a.CS, 1, false));
         } else {
             tq_s = tq_r;
             td_s = td_r;
@@ -779,6 +793,14 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
         }
         Q8_CHECK(launch_pdl(moe_kernel_for(2, nb), dim3(p.grid), dim3(kMoeThreads), p.smem, s,
                             "q8_moe_gemv down launch", tq_r, td_r, tq_s, td_s, tx_r, tx_s, a));
+    }
+    // ---- launch 3: per token, the partials in ascending expert id, then the shared one
+    {
+        const int64_t n = T * H;
+        const int64_t blocks = std::min<int64_t>(ceil_div(n, 256), (int64_t)dev->sms * 4);
+        Q8_CHECK(launch_pdl(moe_sum_kernel, dim3((unsigned)blocks), dim3(256), 0, s, "q8_moe_gemv sum launch",
+                            idx, static_cast<const float *>(part), y, (int)T, (int)E, (int)top_k, (int)H,
+                            has_shared ? 1 : 0));
     }
     return Q8_OK;
 }
