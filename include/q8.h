@@ -80,9 +80,12 @@ const char *q8_last_cuda_error(void);
 
 /* Synchronises the current device, then returns and clears the sticky device
  * error word of the current device: Q8_OK when no kernel recorded a problem,
- * Q8_ERR_DEVICE_TIMEOUT when some kernel's bounded wait ran out (the kernel
- * then returned early and its outputs are incomplete).  *detail (nullable)
- * receives the raw word. */
+ * Q8_ERR_DEVICE_TIMEOUT otherwise.  *detail (nullable) receives the raw word,
+ * an OR of: 1 = a bounded wait ran out (the kernel returned early and its
+ * outputs are incomplete), 2 = waiting for in-flight copies at exit ran out,
+ * 4 = q8_moe_gemv skipped an expert pick (out of range, or repeated within a
+ * token), 8 = a kernel found its launch configuration differing from its
+ * plan (it returned without computing). */
 q8_status q8_read_device_error(uint32_t *detail);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
@@ -160,32 +163,46 @@ q8_status q8_moe_route(const float *logits, int64_t T, int64_t E, int64_t top_k,
 size_t q8_moe_workspace_bytes(int64_t T, int64_t E, int64_t top_k, int64_t H, int64_t I,
                               int64_t I_shared);
 
+/* Zero-fill workspace_bytes bytes of a MoE workspace (asynchronous on
+ * `stream`).  A workspace must be zero-filled once before its first
+ * q8_moe_gemv call; each call that completes without a device error leaves it
+ * ready for the next one.  After a call that recorded a device error
+ * (q8_read_device_error), zero-fill it again. */
+q8_status q8_moe_workspace_init(void *workspace, size_t workspace_bytes, q8_stream_t stream);
+
 /* y[t] = sum_{s < top_k} w[t][s] * Down_e(SwiGLU(GateUp_e x[t]))  (e = idx[t][s])
  *        + Down_sh(SwiGLU(GateUp_sh x[t]))             (when a shared expert is given)
- * in three launches: one computes SwiGLU(gate_up) for every selected
- * (expert, token) pair and the shared expert, one the down projection of
- * each selected expert for its own tokens, and a small one the weighted sum.
- * The weight launches walk only the selected experts, read only their tokens'
- * activations, and an expert picked by several tokens streams its weights
- * once.  The slot
- * weighting and shared expert follow the router + top-k expert +
- * shared-expert FFN block of "Add Qwen1.5-MoE Q8_0 ... - #144" (PR summary);
- * folding the per-slot launches into one grid follows the routed-expert
- * launch fusion in that PR's conversation.  Every output is summed in a fixed
- * order (routed experts by ascending expert id, then the shared expert), so
- * results are bit-identical from run to run.
+ * in one launch of one CTA per SM.  The CTAs first compute SwiGLU(gate_up) for
+ * every selected (expert, token) pair and the shared expert, then the down
+ * projection of each selected expert for its own tokens, then the weighted
+ * sum; counters in the workspace order the phases between CTAs (a down tile
+ * starts once its expert's SwiGLU rows are all stored; the CTA that stores
+ * an output group's last down tile adds that group up), so the down weights
+ * stream while the last SwiGLU rows are still being finished.  Only the
+ * selected experts' weights are read, each once for all of its tokens, and
+ * only their tokens' activations.  The slot weighting and shared expert
+ * follow the router + top-k expert + shared-expert FFN block of "Add
+ * Qwen1.5-MoE Q8_0 ... - #144" (PR summary); folding the per-slot launches
+ * into one grid follows the routed-expert launch fusion in that PR's
+ * conversation.  Every output is summed in a fixed order (routed experts by
+ * ascending expert id, then the shared expert), so results are bit-identical
+ * from run to run.
  *   gate_up_experts: E consecutive packed matrices [2I][H], each
  *       q8_packed_bytes(2I, H) bytes (gate rows first, as q8_gate_up_swiglu).
  *   down_experts:    E consecutive packed matrices [H][I], each
  *       q8_packed_bytes(H, I) bytes.
  *   shared_gate_up / shared_down: packed [2*I_shared][H] / [H][I_shared], or
  *       both NULL (with I_shared = 0) for no shared expert.
- *   idx, w: [T][top_k] as written by q8_moe_route (trusted device data).
+ *   idx, w: [T][top_k] as written by q8_moe_route.  A pick outside [0, E), or
+ *       a token's repeated pick of one expert, is skipped (it adds nothing)
+ *       and sets bit 4 of the device error word (q8_read_device_error).
  *   x: [T][H] fp32.  y: [T][H] fp32, fully overwritten.
- *   workspace: >= q8_moe_workspace_bytes(...) bytes of device scratch, 16-byte
- *       aligned; its contents on entry do not matter.
+ *   workspace: >= q8_moe_workspace_bytes(...) bytes of device memory, 16-byte
+ *       aligned, zero-filled before its first use (q8_moe_workspace_init) and
+ *       then left to the library; calls that may run at the same time must
+ *       not share one.
  * Limits: 1 <= T <= 16, top_k <= 8, E <= 256, H, I, I_shared multiples of 32,
- * I and I_shared multiples of 8. */
+ * H, I, I_shared <= 65536. */
 q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
                       const void *shared_gate_up, const void *shared_down,
                       const int32_t *idx, const float *w, const float *x, float *y, int64_t T,
@@ -206,9 +223,10 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
  * allocated or freed.
  * The first call on each device looks up the array's device address (with
  * that device current); make that first call before any stream capture.
- * All calls share the one array and it keeps the last call's contents; the
- * kernels write every scratch element before reading it, so nothing needs
- * clearing between calls.  Calls that may run at the same time on the GPU
+ * All calls share the one array.  It starts zero-filled and every call that
+ * completes without a device error leaves it ready for the next; after a
+ * device error the next no-alloc call may compute wrong values, so a process
+ * should treat that error as fatal.  Calls that may run at the same time on the GPU
  * (different streams without an ordering between them) race on the array and
  * must not be issued. */
 q8_status q8_moe_gemv_noalloc(const void *gate_up_experts, const void *down_experts,

@@ -19,7 +19,8 @@ import threading
 __all__ = [
     "Q8Error", "lib_path", "q8_status_string", "q8_last_cuda_error", "q8_read_device_error",
     "q8_version", "q8_packed_bytes", "q8_pack_weights", "q8_unpack_weights", "q8_gemv",
-    "q8_gate_up_swiglu", "q8_moe_route", "q8_moe_workspace_bytes", "q8_moe_gemv",
+    "q8_gate_up_swiglu", "q8_moe_route", "q8_moe_workspace_bytes", "q8_moe_workspace_init",
+    "q8_moe_gemv",
     "q8_moe_gemv_noalloc",
     "q8_quantize_act", "q8q8_gemv", "q8q8_block_dots",
 ]
@@ -46,6 +47,7 @@ _SIGS = {
     "q8_gate_up_swiglu": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "q8_moe_route": (_INT, [_P, _I64, _I64, _I64, _INT, _P, _P, _P]),
     "q8_moe_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64, _I64, _I64]),
+    "q8_moe_workspace_init": (_INT, [_P, _SZ, _P]),
     "q8_moe_gemv": (_INT, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64,
                            _P, _SZ, _P]),
     "q8_moe_gemv_noalloc": (_INT, [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64,
@@ -159,6 +161,10 @@ def q8_moe_route(logits, T, E, top_k, renormalize, idx, w, stream=None):
 
 def q8_moe_workspace_bytes(T, E, top_k, H, I, I_shared) -> int:
     return int(_load().q8_moe_workspace_bytes(T, E, top_k, H, I, I_shared))
+
+
+def q8_moe_workspace_init(workspace, workspace_bytes, stream=None):
+    _call("q8_moe_workspace_init", _ptr(workspace), int(workspace_bytes), _stream(stream))
 
 
 def q8_moe_gemv(gate_up_experts, down_experts, shared_gate_up, shared_down, idx, w, x, y, T, E,

@@ -414,97 +414,82 @@ static q8_status run_mma(const void *W, const int8_t *xq, const uint16_t *xd, fl
 // ---------------------------------------------------------------------------
 // grouped MoE (S6)
 // ---------------------------------------------------------------------------
-using MoeKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
-                           CUtensorMap, MoeArgs);
+using MoeKernel = void (*)(MoeMaps, MoeArgs);
 
-// Items per tile: as many as ~32 KB of weights hold at 32 columns a stage
-// (3 gate|up items, 7 down items), and at most 32 fp32 accumulators per lane
-// (items x halves x tokens).  The kernel computes exactly this many, so a
-// full tile wastes nothing.
-__host__ __device__ constexpr int moe_tgm_c(int stage, int nmax) {
-    return stage == 1 ? (16 / nmax < 1 ? 1 : 16 / nmax < 3 ? 16 / nmax : 3)
-                      : (32 / nmax < 7 ? 32 / nmax : 7);
-}
-
-template <int STAGE, int NMAX>
-static MoeKernel moe_kernel_ptr() {
-    return &moe_kernel<STAGE, NMAX, moe_tgm_c(STAGE, NMAX)>;
-}
-
-static int moe_tgm(int stage, int nmax) { return moe_tgm_c(stage, nmax); }
-
-static MoeKernel moe_kernel_for(int stage, int nmax) {
+static MoeKernel moe_kernel_for(int nmax) {
     switch (nmax) {
-        case 1: return stage == 1 ? moe_kernel_ptr<1, 1>() : moe_kernel_ptr<2, 1>();
-        case 2: return stage == 1 ? moe_kernel_ptr<1, 2>() : moe_kernel_ptr<2, 2>();
-        case 4: return stage == 1 ? moe_kernel_ptr<1, 4>() : moe_kernel_ptr<2, 4>();
-        case 8: return stage == 1 ? moe_kernel_ptr<1, 8>() : moe_kernel_ptr<2, 8>();
-        default: return stage == 1 ? moe_kernel_ptr<1, 16>() : moe_kernel_ptr<2, 16>();
+        case 1: return &moe_fused_kernel<1>;
+        case 2: return &moe_fused_kernel<2>;
+        case 4: return &moe_fused_kernel<4>;
+        case 8: return &moe_fused_kernel<8>;
+        default: return &moe_fused_kernel<16>;
     }
 }
 
 static cudaError_t setup_moe_kernels(int max_smem) {
     const int nm[5] = {1, 2, 4, 8, 16};
-    for (int i = 0; i < 5; ++i)
-        for (int stage = 1; stage <= 2; ++stage) {
-            const void *k = reinterpret_cast<const void *>(moe_kernel_for(stage, nm[i]));
-            cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-            if (e != cudaSuccess) return e;
-            e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                     cudaSharedmemCarveoutMaxShared);
-            if (e != cudaSuccess) return e;
-        }
+    for (int i = 0; i < 5; ++i) {
+        const void *k = reinterpret_cast<const void *>(moe_kernel_for(nm[i]));
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+    }
     return cudaSuccess;
 }
 static RegisterSetup g_reg_moe(setup_moe_kernels);
 
 struct MoePlan {
     MoeArgs a;
-    int grid;
     size_t smem;
 };
 
-// Stage shape for a MoE weight launch: TG items of `halves` weight boxes of
-// CS columns (about 32 KB of weights) and one activation box per token of the
-// segment (T at most).  These launches cannot prefetch weights before their
-// dependency wait (the router picks them), so the ring takes most of the
-// SM's shared memory to keep several stages in flight.
-static MoePlan plan_moe(int stage, int64_t T, int64_t c_min, int nmax, int64_t units_bound, int sms) {
-    MoePlan p;
+// Ring slots of the largest stage any tile of this token bucket has; as many
+// as fit next to the barriers, the partial-sum buffers and the table.
+static bool plan_moe(int64_t T, int max_smem, MoePlan &p) {
     MoeArgs &a = p.a;
     a = MoeArgs{};
-    const int halves = stage == 1 ? 2 : 1;
-    p.grid = (int)std::max<int64_t>(1, std::min<int64_t>(sms, units_bound));
-    const int64_t upc = ceil_div(units_bound, p.grid);
-    // 32 columns (8 quads: one per consumer warp) unless K or the activation
-    // boxes are smaller; then as many items as keep ~32 KB of weights a stage
-    int64_t cs = std::min<int64_t>(32, round_up(c_min, 16));
-    const int64_t cs_x = (32 * 1024) / (T * 64) / 16 * 16;
-    cs = std::max<int64_t>(16, std::min<int64_t>(cs, cs_x));
-    const int64_t tg_bytes = std::max<int64_t>(1, (32 * 1024) / (halves * cs * 136));
-    const int tg = (int)std::min<int64_t>(std::min<int64_t>(moe_tgm(stage, nmax), upc), tg_bytes);
-    a.TG = tg;
-    a.CS = (int)cs;
-    a.q_box = (uint32_t)(cs * kColBytes);
-    a.d_box = (uint32_t)(cs * 8);
-    a.x_row = (uint32_t)(cs * 64);
-    a.q_half = (uint32_t)tg * a.q_box;
-    a.d_off = halves * a.q_half;
-    a.d_half = (uint32_t)tg * a.d_box;
-    a.x_off = a.d_off + halves * a.d_half;
-    a.stage_bytes = (uint32_t)round_up(a.x_off + T * a.x_row, 128);
-    const size_t fixed =
-        sizeof(MoeTable) + (size_t)kMoeWarps * moe_tgm(stage, nmax) * halves * nmax * 8 * 4 + 16;
-    const int64_t stages = (int64_t)(190 * 1024 - fixed) / a.stage_bytes;
-    a.stages = (int)(stages < 2 ? 2 : stages > 8 ? 8 : stages);
-    p.smem = (size_t)a.stages * a.stage_bytes + 16 * a.stages + fixed;
-    return p;
+    const int nmax = nmax_for(T);
+    uint32_t slot = 0;
+    int red_a = 0;
+    for (int nx = 1; nx <= nmax; nx *= 2)
+        for (int ph = 1; ph <= 2; ++ph) {
+            slot = std::max(slot, moe_stage_bytes(ph, nx));
+            red_a = std::max(red_a, moe_halves(ph) * moe_tg(ph, nx) * nx);
+        }
+    a.slot_bytes = (uint32_t)round_up(slot, 128);
+    a.red_a = red_a;
+    const size_t fixed = kMoeBarBytes + (size_t)kMoeRedBufs * 8 * red_a * 8 * 4 + sizeof(MoeTable) + 16;
+    const int64_t stages = ((int64_t)max_smem - (int64_t)fixed) / a.slot_bytes;
+    if (stages < 2) return false;
+    a.stages = (int)std::min<int64_t>(stages, kMoeMaxStages);
+    p.smem = (size_t)a.stages * a.slot_bytes + fixed;
+    return true;
 }
 
+// workspace: counters | routed h | shared h | partial outputs
+static size_t moe_ctr_bytes(int64_t H) { return (size_t)round_up((kCtrGroups + H / 8) * 4, 256); }
 static size_t moe_hbuf_bytes(int64_t T, int64_t k, int64_t I) { return (size_t)round_up(T * k * I * 4, 256); }
 static size_t moe_hsh_bytes(int64_t T, int64_t Is) { return (size_t)round_up(T * Is * 4, 256); }
-// launch 2's partial outputs: one row per (token, slot) pair, then one per token
-static size_t moe_part_bytes(int64_t T, int64_t k, int64_t H) { return (size_t)round_up((T * k + T) * H * 4, 256); }
+// K chunks of the shared expert's down projection: about as long as a routed
+// expert's K (at most kMoeMaxSplit chunks), an even number of 16-byte columns
+// each (whole Q8_0 blocks)
+static void moe_shared_chunks(int64_t I, int64_t Is, int &nsplit, int &cc) {
+    if (Is <= 0) {
+        nsplit = 0;
+        cc = 0;
+        return;
+    }
+    const int64_t C = Is / 16, n0 = std::min<int64_t>(ceil_div(Is, I), kMoeMaxSplit);
+    cc = (int)round_up(ceil_div(C, n0), 2);
+    nsplit = (int)ceil_div(C, cc);
+}
+// partial outputs: one row per (token, slot) pair, then one per (shared chunk, token)
+static size_t moe_part_bytes(int64_t T, int64_t k, int64_t H, int64_t I, int64_t Is) {
+    int nsplit, cc;
+    moe_shared_chunks(I, Is, nsplit, cc);
+    return (size_t)round_up((T * k + nsplit * T) * H * 4, 256);
+}
 
 // ---------------------------------------------------------------------------
 // scratch for q8_moe_gemv_noalloc: a fixed array in the library's own device
@@ -692,7 +677,15 @@ q8_status q8_moe_route(const float *logits, int64_t T, int64_t E, int64_t top_k,
 size_t q8_moe_workspace_bytes(int64_t T, int64_t E, int64_t top_k, int64_t H, int64_t I,
                               int64_t I_shared) {
     if (T <= 0 || E <= 0 || top_k <= 0 || H <= 0 || I <= 0 || I_shared < 0) return 0;
-    return moe_hbuf_bytes(T, top_k, I) + moe_hsh_bytes(T, I_shared) + moe_part_bytes(T, top_k, H);
+    return moe_ctr_bytes(H) + moe_hbuf_bytes(T, top_k, I) + moe_hsh_bytes(T, I_shared) +
+           moe_part_bytes(T, top_k, H, I, I_shared);
+}
+
+q8_status q8_moe_workspace_init(void *workspace, size_t workspace_bytes, q8_stream_t stream) {
+    if (workspace_bytes == 0) return Q8_ERR_SHAPE;
+    Q8_CHECK(check_device_ptr(workspace));
+    Q8_CUDA_TRY(cudaMemsetAsync(workspace, 0, workspace_bytes, (cudaStream_t)stream));
+    return Q8_OK;
 }
 
 q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
@@ -724,85 +717,78 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
     if (workspace_bytes < q8_moe_workspace_bytes(T, E, top_k, H, I, I_shared)) return Q8_ERR_SHAPE;
     const DeviceInfo *dev = nullptr;
     Q8_CHECK(device_info(&dev));
-    cudaStream_t s = (cudaStream_t)stream;
-    float *hbuf = static_cast<float *>(workspace);
-    float *hsh = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + moe_hbuf_bytes(T, top_k, I));
-    float *part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + moe_hbuf_bytes(T, top_k, I) +
-                                            moe_hsh_bytes(T, I_shared));
-    const int nb = nmax_for(T);
+    MoePlan p;
+    if (!plan_moe(T, dev->max_smem_optin, p)) return Q8_ERR_UNSUPPORTED;
+    MoeArgs &a = p.a;
     const int64_t Ish = has_shared ? I_shared : 0;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    a.T = (int)T; a.E = (int)E; a.k = (int)top_k; a.H = (int)H; a.I = (int)I; a.Is = (int)Ish;
+    moe_shared_chunks(I, Ish, a.nsplit, a.cc);
+    a.idx = idx;
+    a.w = w;
+    a.y = y;
+    a.ctr = reinterpret_cast<unsigned *>(ws);
+    a.hbuf = reinterpret_cast<float *>(ws + moe_ctr_bytes(H));
+    a.hsh = reinterpret_cast<float *>(ws + moe_ctr_bytes(H) + moe_hbuf_bytes(T, top_k, I));
+    a.part = reinterpret_cast<float *>(ws + moe_ctr_bytes(H) + moe_hbuf_bytes(T, top_k, I) +
+                                       moe_hsh_bytes(T, I_shared));
 
-    // ---- launch 1: gate_up + SwiGLU over selected experts and the shared one
-    {
-        const int64_t units_bound = std::min<int64_t>(T * top_k, E) * (I / 8) + Ish / 8;
-        MoePlan p = plan_moe(1, T, H / 16, nb, units_bound, dev->sms);
-        MoeArgs &a = p.a;
-        a.T = (int)T; a.E = (int)E; a.k = (int)top_k; a.H = (int)H; a.I = (int)I; a.Is = (int)Ish;
-        a.idx = idx; a.w = w; a.hbuf = hbuf; a.hsh = hsh; a.part = part; a.y = y;
-        if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
-        const uint64_t gs = (uint64_t)kGroupBytesPerBlock * (H / 32);
-        CUtensorMap tq_r, td_r, tq_s, td_s, tx;
-        Q8_CHECK(make_map_3d(&tq_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, gate_up_experts, kColBytes, H / 16,
-                             E * (2 * I / 8), kColBytes, gs, kColBytes, a.CS, 1, true));
-        Q8_CHECK(make_map_3d(&td_r, CU_TENSOR_MAP_DATA_TYPE_UINT16,
-                             static_cast<const uint8_t *>(gate_up_experts) + 256 * (H / 32), 8, H / 32,
-                             E * (2 * I / 8), 16, gs, 8, a.CS / 2, 1, true));
-        const void *sgu = has_shared ? shared_gate_up : gate_up_experts;
-        const int64_t sg = has_shared ? 2 * Ish / 8 : E * (2 * I / 8);
-        Q8_CHECK(make_map_3d(&tq_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, sgu, kColBytes, H / 16, sg, kColBytes, gs,
-                             kColBytes, a.CS, 1, true));
-        Q8_CHECK(make_map_3d(&td_s, CU_TENSOR_MAP_DATA_TYPE_UINT16,
-                             static_cast<const uint8_t *>(sgu) + 256 * (H / 32), 8, H / 32, sg, 16, gs, 8,
-                             a.CS / 2, 1, true));
-        Q8_CHECK(make_map_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, H / 16, T, 64, (uint64_t)H * 4, 16,
-                             a.CS, 1, false));
-        Q8_CHECK(launch_pdl(moe_kernel_for(1, nb), dim3(p.grid), dim3(kMoeThreads), p.smem, s,
-                            "q8_moe_gemv gate_up launch", tq_r, td_r, tq_s, td_s, tx, tx, a));
+    // Weight maps: [16-byte column][8 rows x 16 B] q boxes and [block][8 rows]
+    // fp16 scale boxes of one packed group each (the tile kernels' maps).
+    // Activation maps: [row][column][16 fp32], one row per box, or all T rows
+    // for the shared expert's segment.
+    MoeMaps m;
+    const uint64_t gs1 = (uint64_t)kGroupBytesPerBlock * (H / 32);
+    const uint64_t gs2 = (uint64_t)kGroupBytesPerBlock * (I / 32);
+    const uint8_t *gu = static_cast<const uint8_t *>(gate_up_experts);
+    const uint8_t *dn = static_cast<const uint8_t *>(down_experts);
+    for (int deep = 0; deep < 2; ++deep) {
+        const uint32_t b1 = deep ? kMoeTile1 : 1, b2 = deep ? kMoeTile2 : 1;
+        Q8_CHECK(make_map_3d(deep ? &m.q1r_t : &m.q1r, CU_TENSOR_MAP_DATA_TYPE_UINT8, gu, kColBytes, H / 16,
+                             E * (2 * I / 8), kColBytes, gs1, kColBytes, kMoeCS, b1, true));
+        Q8_CHECK(make_map_3d(deep ? &m.d1r_t : &m.d1r, CU_TENSOR_MAP_DATA_TYPE_UINT16, gu + 256 * (H / 32), 8,
+                             H / 32, E * (2 * I / 8), 16, gs1, 8, kMoeCS / 2, b1, true));
+        Q8_CHECK(make_map_3d(deep ? &m.q2r_t : &m.q2r, CU_TENSOR_MAP_DATA_TYPE_UINT8, dn, kColBytes, I / 16,
+                             E * (H / 8), kColBytes, gs2, kColBytes, kMoeCS, b2, true));
+        Q8_CHECK(make_map_3d(deep ? &m.d2r_t : &m.d2r, CU_TENSOR_MAP_DATA_TYPE_UINT16, dn + 256 * (I / 32), 8,
+                             I / 32, E * (H / 8), 16, gs2, 8, kMoeCS / 2, b2, true));
     }
-    // ---- launch 2: down projection of each selected expert for its tokens
-    {
-        const int64_t c_min = has_shared ? std::min<int64_t>(I, Ish) / 16 : I / 16;
-        const int64_t units_bound = (std::min<int64_t>(T * top_k, E) + (has_shared ? 1 : 0)) * (H / 8);
-        MoePlan p = plan_moe(2, T, c_min, nb, units_bound, dev->sms);
-        MoeArgs &a = p.a;
-        a.T = (int)T; a.E = (int)E; a.k = (int)top_k; a.H = (int)H; a.I = (int)I; a.Is = (int)Ish;
-        a.idx = idx; a.w = w; a.hbuf = hbuf; a.hsh = hsh; a.part = part; a.y = y;
-        if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
-        const uint64_t gs_r = (uint64_t)kGroupBytesPerBlock * (I / 32);
-        CUtensorMap tq_r, td_r, tq_s, td_s, tx_r, tx_s;
-        Q8_CHECK(make_map_3d(&tq_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, down_experts, kColBytes, I / 16,
-                             E * (H / 8), kColBytes, gs_r, kColBytes, a.CS, 1, true));
-        Q8_CHECK(make_map_3d(&td_r, CU_TENSOR_MAP_DATA_TYPE_UINT16,
-                             static_cast<const uint8_t *>(down_experts) + 256 * (I / 32), 8, I / 32,
-                             E * (H / 8), 16, gs_r, 8, a.CS / 2, 1, true));
-        Q8_CHECK(make_map_3d(&tx_r, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, hbuf, 16, I / 16, T * top_k, 64,
-                             (uint64_t)I * 4, 16, a.CS, 1, false));
-        if (has_shared) {
-            const uint64_t gs_s = (uint64_t)kGroupBytesPerBlock * (Ish / 32);
-            Q8_CHECK(make_map_3d(&tq_s, CU_TENSOR_MAP_DATA_TYPE_UINT8, shared_down, kColBytes, Ish / 16, H / 8,
-                                 kColBytes, gs_s, kColBytes, a.CS, 1, true));
-            Q8_CHECK(make_map_3d(&td_s, CU_TENSOR_MAP_DATA_TYPE_UINT16,
-                                 static_cast<const uint8_t *>(shared_down) + 256 * (Ish / 32), 8, Ish / 32,
-                                 H / 8, 16, gs_s, 8, a.CS / 2, 1, true));
-            Q8_CHECK(make_map_3d(&tx_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, hsh, 16, Ish / 16, T, 64,
-                                 (uint64_t)Ish * 4, 16, a.CS, 1, false));
-        } else {
-            tq_s = tq_r;
-            td_s = td_r;
-            tx_s = tx_r;
+    Q8_CHECK(make_map_3d(&m.x1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, H / 16, T, 64, (uint64_t)H * 4, 16, kMoeCS,
+                         1, false));
+    Q8_CHECK(make_map_3d(&m.x1s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, H / 16, T, 64, (uint64_t)H * 4, 16, kMoeCS,
+                         (uint32_t)T, false));
+    Q8_CHECK(make_map_3d(&m.h2r, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.hbuf, 16, I / 16, T * top_k, 64,
+                         (uint64_t)I * 4, 16, kMoeCS, 1, false));
+    if (has_shared) {
+        const uint64_t gss = (uint64_t)kGroupBytesPerBlock * (Ish / 32);
+        const uint8_t *sgu = static_cast<const uint8_t *>(shared_gate_up);
+        const uint8_t *sdn = static_cast<const uint8_t *>(shared_down);
+        for (int deep = 0; deep < 2; ++deep) {
+            const uint32_t b1 = deep ? kMoeTile1 : 1, b2 = deep ? kMoeTile2 : 1;
+            Q8_CHECK(make_map_3d(deep ? &m.q1s_t : &m.q1s, CU_TENSOR_MAP_DATA_TYPE_UINT8, sgu, kColBytes, H / 16,
+                                 2 * Ish / 8, kColBytes, gs1, kColBytes, kMoeCS, b1, true));
+            Q8_CHECK(make_map_3d(deep ? &m.d1s_t : &m.d1s, CU_TENSOR_MAP_DATA_TYPE_UINT16, sgu + 256 * (H / 32), 8,
+                                 H / 32, 2 * Ish / 8, 16, gs1, 8, kMoeCS / 2, b1, true));
+            Q8_CHECK(make_map_3d(deep ? &m.q2s_t : &m.q2s, CU_TENSOR_MAP_DATA_TYPE_UINT8, sdn, kColBytes, Ish / 16,
+                                 H / 8, kColBytes, gss, kColBytes, kMoeCS, b2, true));
+            Q8_CHECK(make_map_3d(deep ? &m.d2s_t : &m.d2s, CU_TENSOR_MAP_DATA_TYPE_UINT16, sdn + 256 * (Ish / 32), 8,
+                                 Ish / 32, H / 8, 16, gss, 8, kMoeCS / 2, b2, true));
         }
-        Q8_CHECK(launch_pdl(moe_kernel_for(2, nb), dim3(p.grid), dim3(kMoeThreads), p.smem, s,
-                            "q8_moe_gemv down launch", tq_r, td_r, tq_s, td_s, tx_r, tx_s, a));
+        Q8_CHECK(make_map_3d(&m.h2s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.hsh, 16, Ish / 16, T, 64,
+                             (uint64_t)Ish * 4, 16, kMoeCS, (uint32_t)T, false));
+    } else {
+        m.q1s = m.q1r;
+        m.d1s = m.d1r;
+        m.q2s = m.q2r;
+        m.d2s = m.d2r;
+        m.q1s_t = m.q1r_t;
+        m.d1s_t = m.d1r_t;
+        m.q2s_t = m.q2r_t;
+        m.d2s_t = m.d2r_t;
+        m.h2s = m.h2r;
     }
-    // ---- launch 3: per token, the partials in ascending expert id, then the shared one
-    {
-        const int64_t n = T * H;
-        const int64_t blocks = std::min<int64_t>(ceil_div(n, 256), (int64_t)dev->sms * 4);
-        Q8_CHECK(launch_pdl(moe_sum_kernel, dim3((unsigned)blocks), dim3(256), 0, s, "q8_moe_gemv sum launch",
-                            idx, static_cast<const float *>(part), y, (int)T, (int)E, (int)top_k, (int)H,
-                            has_shared ? 1 : 0));
-    }
-    return Q8_OK;
+    return launch_pdl(moe_kernel_for(nmax_for(T)), dim3((unsigned)dev->sms), dim3(moe_threads(nmax_for(T))), p.smem,
+                      (cudaStream_t)stream, "q8_moe_gemv launch", m, a);
 }
 
 q8_status q8_moe_gemv_noalloc(const void *gate_up_experts, const void *down_experts,
@@ -821,8 +807,8 @@ q8_status q8_moe_gemv_noalloc(const void *gate_up_experts, const void *down_expe
     }
     void *scratch = nullptr;
     Q8_CHECK(moe_noalloc_scratch(&scratch));
-    // The MoE launches write every scratch element before they read it, so the
-    // previous call's contents never need clearing.
+    // The array starts zero-filled (a static device array) and every call
+    // leaves its counters zero again, as the MoE kernel requires.
     return q8_moe_gemv(gate_up_experts, down_experts, shared_gate_up, shared_down, idx, w, x, y, T,
                        E, top_k, H, I, I_shared, scratch, need, stream);
 }

@@ -2,6 +2,7 @@
 
     python -m q8_block_quantized_02_b200.profile --op gemv --M 151936 --K 896 --N 1
     python -m q8_block_quantized_02_b200.profile --op q8q8 --M 37888 --K 3584 --N 16
+    python -m q8_block_quantized_02_b200.profile --op moe --T 1
 
 Weights follow the synthetic Q8_0 recipe (q uniform in [-127, 127], d =
 |N(0,1)| * 0.02) and activations are N(0,1).  Enough packed copies of the
@@ -14,6 +15,15 @@ bytes (34 per 32 weights) per second.
 
 This is also the driver for ncu captures of a single kernel: with
 `--copies 1 --reps 3 --warmup 2` it makes five launches on one matrix.
+
+`--op moe` times q8_moe_gemv on Qwen1.5-MoE-A2.7B shapes (60 experts of
+gate_up 2816 x 2048 and down 2048 x 1408, a shared expert of intermediate
+5632, top-4; all sizes can be changed).  All experts are packed once
+(about 590 MB, more than L2).  `--routings` sets of router logits ~ N(0,1)
+are routed up front (q8_moe_route, not timed) and the timed calls cycle
+through them, so consecutive calls select different experts.  Bytes per
+call count each call's distinct selected experts plus the shared expert once
+(34 B per 32 weights).
 """
 from __future__ import annotations
 
@@ -29,7 +39,7 @@ if ROOT not in sys.path:
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--op", choices=["gemv", "swiglu", "q8q8"], default="gemv",
+    ap.add_argument("--op", choices=["gemv", "swiglu", "q8q8", "moe"], default="gemv",
                     help="q8_gemv, q8_gate_up_swiglu (M = rows of the stacked gate|up matrix) "
                          "or q8_quantize_act + q8q8_gemv (only q8q8_gemv is timed)")
     ap.add_argument("--M", type=int, default=151936)
@@ -39,7 +49,16 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--copies", type=int, default=0, help="packed weight copies (0: cover 3x L2)")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--T", type=int, default=1, help="moe: tokens")
+    ap.add_argument("--E", type=int, default=60, help="moe: routed experts")
+    ap.add_argument("--H", type=int, default=2048, help="moe: hidden size")
+    ap.add_argument("--I", type=int, default=1408, help="moe: expert intermediate size")
+    ap.add_argument("--Is", type=int, default=5632, help="moe: shared expert intermediate size (0: none)")
+    ap.add_argument("--k", type=int, default=4, help="moe: experts per token")
+    ap.add_argument("--routings", type=int, default=16, help="moe: distinct routings cycled through")
     args = ap.parse_args(argv)
+    if args.op == "moe":
+        return _moe(args)
 
     import numpy as np
     import torch
@@ -99,6 +118,72 @@ def main(argv=None) -> int:
     weight_bytes = M * K * 34 // 32
     print(json.dumps({"op": args.op, "M": M, "K": K, "N": N, "us_per_call": round(us, 3),
                       "weight_GBps": round(weight_bytes / (us * 1e-6) / 1e9, 1), "copies": copies,
+                      "reps": args.reps, "device_error": word}), flush=True)
+    return 0 if st == 0 else 1
+
+
+def _moe(args) -> int:
+    import numpy as np
+    import torch
+
+    import q8gen
+    import q8_block_quantized_02_b200 as q8
+
+    T, E, H, I, Is, k = args.T, args.E, args.H, args.I, args.Is, args.k
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    def stack(seed0, n, M, K):
+        one = q8.q8_packed_bytes(M, K)
+        out = torch.empty(n * one, dtype=torch.uint8, device=dev)
+        for e in range(n):
+            g, _ = q8gen.q8_matrix(seed0 + e, M, K)
+            q8.q8_pack_weights(torch.from_numpy(g).to(dev), M, K, out[e * one:(e + 1) * one])
+        return out
+
+    p_gu, p_dn = stack(args.seed, E, 2 * I, H), stack(args.seed + 1000, E, H, I)
+    p_sgu = p_sdn = None
+    if Is:
+        p_sgu, p_sdn = stack(args.seed + 2000, 1, 2 * Is, H), stack(args.seed + 2001, 1, H, Is)
+    R = max(1, args.routings)
+    idx = torch.empty((R, T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((R, T, k), dtype=torch.float32, device=dev)
+    for r in range(R):
+        lg = torch.from_numpy(q8gen.logits(args.seed + 100 + r, T, E)).to(dev)
+        q8.q8_moe_route(lg, T, E, k, 0, idx[r], w[r])
+    x = torch.from_numpy(q8gen.activations(args.seed + 7, T, H)).to(dev)
+    y = torch.empty((T, H), dtype=torch.float32, device=dev)
+    ws_bytes = q8.q8_moe_workspace_bytes(T, E, k, H, I, Is)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    q8.q8_moe_workspace_init(ws, ws_bytes)
+    it = [0]
+
+    def call():
+        r = it[0] % R
+        it[0] += 1
+        q8.q8_moe_gemv(p_gu, p_dn, p_sgu, p_sdn, idx[r], w[r], x, y, T, E, k, H, I, Is, ws, ws_bytes)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    start = it[0]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.reps):
+        call()
+    t1.record()
+    torch.cuda.synchronize()
+    st, word = q8.q8_read_device_error()
+    us = t0.elapsed_time(t1) * 1e3 / max(1, args.reps)
+    per_expert = (2 * I * H + H * I) * 34 // 32
+    shared = (2 * Is * H + H * Is) * 34 // 32
+    picks = idx.cpu().numpy()
+    uniq = [len(np.unique(picks[(start + i) % R])) for i in range(args.reps)]
+    mean_bytes = float(np.mean(uniq)) * per_expert + shared
+    print(json.dumps({"op": "moe", "T": T, "E": E, "H": H, "I": I, "Is": Is, "k": k,
+                      "us_per_call": round(us, 3), "unique_experts": round(float(np.mean(uniq)), 2),
+                      "weight_MB": round(mean_bytes / 1e6, 2),
+                      "weight_GBps": round(mean_bytes / (us * 1e-6) / 1e9, 1), "routings": R,
                       "reps": args.reps, "device_error": word}), flush=True)
     return 0 if st == 0 else 1
 

@@ -33,7 +33,8 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     for required in ("q8_pack_weights", "q8_gemv", "q8_gate_up_swiglu", "q8_moe_route",
                      "q8_moe_gemv", "q8_quantize_act", "q8q8_gemv", "q8q8_block_dots",
-                     "q8_packed_bytes", "q8_moe_workspace_bytes", "q8_unpack_weights"):
+                     "q8_packed_bytes", "q8_moe_workspace_bytes", "q8_moe_workspace_init",
+                     "q8_unpack_weights"):
         assert required in names
 
 

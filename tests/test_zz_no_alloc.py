@@ -58,6 +58,7 @@ def test_noalloc_matches_workspace_entry_point():
 
         ws_bytes = q8.q8_moe_workspace_bytes(T, E, k, H, I, Is)
         ws = t.empty(ws_bytes, dtype=t.uint8, device="cuda")
+        q8.q8_moe_workspace_init(ws, ws_bytes)
         y_ws = t.full((T, H), float("nan"), dtype=t.float32, device="cuda")
         q8.q8_moe_gemv(p_gu, p_dn, p_sgu, p_sdn, idx, w, xd, y_ws, T, E, k, H, I, Is, ws, ws_bytes)
 
