@@ -23,14 +23,15 @@
 //     group's last phase-2 item (a counter per group says which one).
 //
 // A selected expert's weights stream once for all of its tokens, and nothing
-// else is read.  One CTA runs per SM.  CTA c owns balanced slices of three
-// lists, walked in this order: the shared expert's phase-1 items (known
-// before the router's output is), the routed phase-1 items, and the phase-2
-// items (shared, then routed, balanced by length).  So the shared expert's
-// gate/up weights are requested before griddepcontrol.wait and stream while
-// the previous kernel on the stream finishes, and phase-2 weights stream into
-// free ring slots while the h they multiply is still being finished by other
-// CTAs.
+// else is read.  One CTA runs per SM.  CTA c owns an even slice of each of
+// four lists, walked in this order: the shared expert's phase-1 items (known
+// before the router's output is), the routed phase-1 items, the shared
+// expert's phase-2 items and the routed phase-2 items.  So the shared
+// expert's gate/up weights are requested before griddepcontrol.wait and
+// stream while the previous kernel on the stream finishes; every CTA's first
+// phase-2 items multiply the shared expert's h, which is complete first; and
+// phase-2 weights stream into free ring slots while the h they multiply is
+// still being finished by other CTAs.
 //
 // Warp roles (CW + 3 warps):
 //   * warps 0..CW-1 consume.  Warp w takes column quad w & 7 of every stage
@@ -93,11 +94,12 @@ constexpr int kCtrGroups = kCtrRouted + kMoeMaxSeg;  // phase-2 segments done, o
 __host__ __device__ constexpr int moe_nx(int cnt) {
     return cnt <= 1 ? 1 : cnt <= 2 ? 2 : cnt <= 4 ? 4 : cnt <= 8 ? 8 : 16;
 }
-// Items per tile: 8 (phase 1: 4 gate|up pairs) for up to 4 tokens, a stage of
-// about 36 KB of weights; fewer for 8 and 16 tokens, so that a lane holds at
-// most 32 accumulators (its items x halves x tokens).
+// Items per tile: 8 down items, or 6 gate|up pairs for up to two tokens (one
+// token's gate/up slice of about 5 items stays one tile), 4 for four tokens;
+// fewer for 8 and 16 tokens, so that a lane holds at most 32 accumulators
+// (its items x halves x tokens).
 __host__ __device__ constexpr int moe_tg(int phase, int nx) {
-    return (phase == 1 ? 4 : 8) / (nx <= 4 ? 1 : nx / 4);
+    return phase == 1 ? (nx <= 2 ? 6 : nx <= 4 ? 4 : 16 / nx) : (nx <= 4 ? 8 : 32 / nx);
 }
 __host__ __device__ constexpr int moe_halves(int phase) { return phase == 1 ? 2 : 1; }
 constexpr int kMoeTile1 = moe_tg(1, 1), kMoeTile2 = moe_tg(2, 1);  // the largest tiles
@@ -325,44 +327,38 @@ __device__ __forceinline__ void moe_build_table_t1(MoeTable &tb, const MoeArgs &
 struct MoeRanges {
     int s0, s1;   // phase-1 shared items
     int r0, r1;   // phase-1 routed items, flattened segment-major (I/8 per segment)
-    int q0, q1;   // phase-2 items: [0, S2) shared (chunk-major), then routed flattened (H/8 per segment)
-    int S2;       // phase-2 shared items (nsplit * H/8)
-    bool table;   // r*, q* are set
+    int q0, q1;   // phase-2 shared items, chunk-major (H/8 per chunk)
+    int v0, v1;   // phase-2 routed items, flattened segment-major (H/8 per segment)
+    bool table;   // r*, q*, v* are set
 };
 
-// The shared expert's phase-1 items split evenly: known without idx.
+// The shared expert's items split evenly: known without idx.
 __device__ __forceinline__ MoeRanges moe_ranges_shared(const MoeArgs &a) {
     MoeRanges rg{};
-    const long long S1 = a.Is / kGroupRows;
+    const long long S1 = a.Is / kGroupRows, S2 = (long long)a.nsplit * (a.H / kGroupRows);
     rg.s0 = (int)(S1 * blockIdx.x / gridDim.x);
     rg.s1 = (int)(S1 * (blockIdx.x + 1) / gridDim.x);
+    rg.q0 = (int)(S2 * blockIdx.x / gridDim.x);
+    rg.q1 = (int)(S2 * (blockIdx.x + 1) / gridDim.x);
     rg.table = false;
     return rg;
 }
 
-// Phase-2 split by length (an item's weight is its stage count): the first
-// item at or after work position W * c / grid.  Monotone in c, 0 at c = 0
-// and the item count at c = grid, so the CTAs' ranges partition the list.
-__device__ __forceinline__ int moe_split2(long long W, long long Ws, int S2, int ks_s, int ks_r, int c,
-                                          int grid) {
-    const long long P = W * c / grid;
-    if (P < Ws) return (int)((P + ks_s - 1) / ks_s);
-    return S2 + (int)((P - Ws + ks_r - 1) / ks_r);
-}
-
+// Each list is split evenly over the CTAs (all of a list's items are equally
+// long), and a CTA walks its slices in list order: shared gate/up (no idx
+// needed), routed gate/up, shared down (its h completes first: every CTA
+// starts with the shared gate/up items), routed down.
 __device__ __forceinline__ void moe_ranges_routed(MoeRanges &rg, const MoeTable &tb, const MoeArgs &a) {
-    const int G = gridDim.x, c = blockIdx.x;
+    const long long G = gridDim.x, c = blockIdx.x;
     const long long R1 = (long long)tb.n_routed * (a.I / kGroupRows);
+    const long long S2 = (long long)a.nsplit * (a.H / kGroupRows);
+    const long long R2 = (long long)tb.n_routed * (a.H / kGroupRows);
     rg.r0 = (int)(R1 * c / G);
     rg.r1 = (int)(R1 * (c + 1) / G);
-    const int S2 = a.nsplit * (a.H / kGroupRows);
-    const int ks_s = a.nsplit > 0 ? (a.cc + kMoeCS - 1) / kMoeCS : 1;
-    const int ks_r = (a.I / 16 + kMoeCS - 1) / kMoeCS;
-    const long long Ws = (long long)S2 * ks_s;
-    const long long W = Ws + (long long)tb.n_routed * (a.H / kGroupRows) * ks_r;
-    rg.S2 = S2;
-    rg.q0 = moe_split2(W, Ws, S2, ks_s, ks_r, c, G);
-    rg.q1 = moe_split2(W, Ws, S2, ks_s, ks_r, c + 1, G);
+    rg.q0 = (int)(S2 * c / G);
+    rg.q1 = (int)(S2 * (c + 1) / G);
+    rg.v0 = (int)(R2 * c / G);
+    rg.v1 = (int)(R2 * (c + 1) / G);
     rg.table = true;
 }
 
@@ -380,7 +376,7 @@ struct MoeTile {
 };
 
 struct MoeCursor {
-    int kind;  // 0: phase-1 shared, 1: phase-1 routed, 2: phase 2, 3: done
+    int kind;  // 0: phase-1 shared, 1: phase-1 routed, 2: phase-2 shared, 3: phase-2 routed, 4: done
     int u;
 };
 
@@ -420,29 +416,34 @@ __device__ __forceinline__ bool moe_next(MoeCursor &cur, const MoeRanges &rg, co
     }
     if (cur.kind == 2) {
         if (cur.u < rg.q1) {
+            const int opg = a.H / kGroupRows;
             t.phase = 2;
-            if (cur.u < rg.S2) {
-                const int opg = a.H / kGroupRows;
-                t.seg = -1;
-                t.split = cur.u / opg;
-                t.in_seg = cur.u - t.split * opg;
-                t.cnt = a.T;
-                t.nx = moe_nx(a.T);
-                t.tga = min(min(moe_tg(2, t.nx), rg.q1 - cur.u), opg - t.in_seg);
-                t.c0 = t.split * a.cc;
-                t.cols = min(a.cc, a.Is / 16 - t.c0);
-            } else {
-                const int opg = a.H / kGroupRows, v = cur.u - rg.S2;
-                t.seg = v / opg;
-                t.in_seg = v - t.seg * opg;
-                t.cnt = tb.seg_cnt[t.seg];
-                t.nx = moe_nx(t.cnt);
-                t.tga = min(min(moe_tg(2, t.nx), rg.q1 - cur.u), opg - t.in_seg);
-                t.cols = a.I / 16;
-            }
+            t.seg = -1;
+            t.split = cur.u / opg;
+            t.in_seg = cur.u - t.split * opg;
+            t.cnt = a.T;
+            t.nx = moe_nx(a.T);
+            t.tga = min(min(moe_tg(2, t.nx), rg.q1 - cur.u), opg - t.in_seg);
+            t.c0 = t.split * a.cc;
+            t.cols = min(a.cc, a.Is / 16 - t.c0);
             goto found;
         }
         cur.kind = 3;
+        cur.u = rg.v0;
+    }
+    if (cur.kind == 3) {
+        if (cur.u < rg.v1) {
+            const int opg = a.H / kGroupRows;
+            t.phase = 2;
+            t.seg = cur.u / opg;
+            t.in_seg = cur.u - t.seg * opg;
+            t.cnt = tb.seg_cnt[t.seg];
+            t.nx = moe_nx(t.cnt);
+            t.tga = min(min(moe_tg(2, t.nx), rg.v1 - cur.u), opg - t.in_seg);
+            t.cols = a.I / 16;
+            goto found;
+        }
+        cur.kind = 4;
     }
     return false;
 found:
@@ -751,54 +752,64 @@ __device__ __forceinline__ void moe_epilogue(MoeTable &tb, const MoeArgs &a, con
 // ---------------------------------------------------------------------------
 // Producers
 // ---------------------------------------------------------------------------
-// Weight maps come in two box depths: one group (any tile) and a full tile's
-// kMoeTile1 / kMoeTile2 consecutive groups, so a full tile takes one box per
-// half instead of one per item.
+// Weight maps: [phase 1 | 2][routed stack | shared][q | scales][box depth
+// 1, 2, 4, 8 groups].  A tile's items are consecutive packed groups, so a
+// stage of tga items takes one box per set bit of tga (and half) instead of
+// one per item: an SM's TMA unit accepts about one instruction per 70 ns,
+// which per-item boxes of 4 KB would make the stream's limit.
+constexpr int kMoeDepths = 4;
 struct MoeMaps {
-    CUtensorMap q1r, d1r, q1s, d1s;   // gate|up weights: routed stack, shared
-    CUtensorMap q2r, d2r, q2s, d2s;   // down weights: routed stack, shared
-    CUtensorMap q1r_t, d1r_t, q1s_t, d1s_t;  // ... box of kMoeTile1 groups
-    CUtensorMap q2r_t, d2r_t, q2s_t, d2s_t;  // ... box of kMoeTile2 groups
+    CUtensorMap w[2][2][2][kMoeDepths];
     CUtensorMap x1, x1s;              // x [T][H]: one token per box, all T tokens per box
     CUtensorMap h2r, h2s;             // routed h [T*k][I] (one pair row per box), shared h [T][Is] (T rows)
 };
 
-// Weight boxes of one tile's stages.  Returns false when a wait failed.
+// Weight boxes of one tile's stages, by the whole warp: lane 0 waits for the
+// slot and arms its barrier, then the lanes issue the boxes in parallel.
+// Returns false (warp-uniform) when a wait failed.
 __device__ __forceinline__ bool moe_issue_weights(uint8_t *smem, const MoeArgs &a, const MoeMaps &m,
                                                   const MoeTable &tb, uint32_t full0, uint32_t empty0,
                                                   volatile int *abort_flag, int &it, const MoeTile &t,
-                                                  uint64_t pw) {
+                                                  uint64_t pw, int lane) {
     const int HH = t.phase == 1 ? 2 : 1, TG = moe_tg(t.phase, t.nx);
     const bool shared = t.seg < 0;
+    // packed group of the tile's first item, and the gate -> up distance
     int g0, up = 0;
-    const CUtensorMap *mq, *md;
-    // a full tile of the deep maps' depth: one box per half
-    const bool deep = t.tga == TG && TG == (t.phase == 1 ? kMoeTile1 : kMoeTile2);
     if (t.phase == 1) {
         const int gates = (shared ? a.Is : a.I) / kGroupRows;
         g0 = (shared ? 0 : tb.seg_expert[t.seg] * 2 * gates) + t.in_seg;
         up = gates;
-        mq = deep ? (shared ? &m.q1s_t : &m.q1r_t) : (shared ? &m.q1s : &m.q1r);
-        md = deep ? (shared ? &m.d1s_t : &m.d1r_t) : (shared ? &m.d1s : &m.d1r);
     } else {
         g0 = (shared ? 0 : tb.seg_expert[t.seg] * (a.H / kGroupRows)) + t.in_seg;
-        mq = deep ? (shared ? &m.q2s_t : &m.q2r_t) : (shared ? &m.q2s : &m.q2r);
-        md = deep ? (shared ? &m.d2s_t : &m.d2r_t) : (shared ? &m.d2s : &m.d2r);
     }
-    const int boxes = deep ? 1 : t.tga;
+    const CUtensorMap(&maps)[2][kMoeDepths] = m.w[t.phase - 1][shared ? 1 : 0];
+    const int bits = __popc(t.tga), per = bits * HH;  // boxes per half, per stage (q; scales alike)
     const uint32_t dbase = (uint32_t)HH * TG * kMoeQBox;
     for (int ks = 0; ks < t.ks_n; ++ks, ++it) {
         const int slot = it % a.stages;
-        if (it >= a.stages && !mbar_wait(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag)) return false;
+        if (it >= a.stages && !mbar_wait_warp(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag))
+            return false;
         const uint32_t st = smem_u32(smem + (size_t)slot * a.slot_bytes);
         const uint32_t full = full0 + 8 * slot;
-        mbar_arrive_expect_tx(full, (uint32_t)(HH * t.tga) * (kMoeQBox + kMoeDBox));
-        for (int g = 0; g < boxes; ++g)
-            for (int h = 0; h < HH; ++h) {
-                const int grp = g0 + g + h * up, b = h * TG + g;
-                tma_load_3d(st + b * kMoeQBox, mq, full, 0, t.c0 + ks * kMoeCS, grp, pw);
-                tma_load_3d(st + dbase + b * kMoeDBox, md, full, 0, (t.c0 >> 1) + ks * (kMoeCS / 2), grp, pw);
-            }
+        if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)(HH * t.tga) * (kMoeQBox + kMoeDBox));
+        __syncwarp();
+        for (int i = lane; i < 2 * per; i += 32) {
+            const bool dbox = i >= per;
+            const int j = dbox ? i - per : i, h = j / bits, k = j - h * bits;
+            // the k-th set bit of tga, from the largest: box depth and first item
+            int d = 3, off = 0, n = 0;
+            for (; d >= 0; --d)
+                if ((t.tga >> d) & 1) {
+                    if (n == k) break;
+                    off += 1 << d;
+                    ++n;
+                }
+            const int grp = g0 + off + h * up, b = h * TG + off;
+            if (dbox)
+                tma_load_3d(st + dbase + b * kMoeDBox, &maps[1][d], full, 0, (t.c0 >> 1) + ks * (kMoeCS / 2), grp, pw);
+            else
+                tma_load_3d(st + b * kMoeQBox, &maps[0][d], full, 0, t.c0 + ks * kMoeCS, grp, pw);
+        }
     }
     return true;
 }
@@ -881,21 +892,20 @@ __global__ void __launch_bounds__(moe_threads(NMAX), 1)
     MoeTile t;
     if (warp == CW) {
         // ------------------------- weight producer -------------------------
-        if (lane == 0) {
+        {
             const uint64_t pw = policy_evict_first();
             int it = 0;
             bool ok = true;
             // the shared expert's gate|up boxes need nothing from earlier kernels
-            while (ok && moe_next(cur, rg, tb, a, t)) ok = moe_issue_weights(smem, a, maps, tb, full0, empty0, abort_flag, it, t, pw);
+            while (ok && moe_next(cur, rg, tb, a, t))
+                ok = moe_issue_weights(smem, a, maps, tb, full0, empty0, abort_flag, it, t, pw, lane);
             pdl_wait_and_trigger();
-            if (ok && mbar_wait(tbl_ready, 0, abort_flag)) {
+            if (ok && mbar_wait_warp(tbl_ready, 0, abort_flag)) {
                 moe_ranges_routed(rg, tb, a);
                 while (ok && moe_next(cur, rg, tb, a, t))
-                    ok = moe_issue_weights(smem, a, maps, tb, full0, empty0, abort_flag, it, t, pw);
+                    ok = moe_issue_weights(smem, a, maps, tb, full0, empty0, abort_flag, it, t, pw, lane);
             }
-            *issued_w = it;
-        } else {
-            pdl_wait_and_trigger();
+            if (lane == 0) *issued_w = it;
         }
     } else if (warp == CW + 1) {
         // ----------------------- activation producer -----------------------

@@ -734,25 +734,26 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
                                        moe_hsh_bytes(T, I_shared));
 
     // Weight maps: [16-byte column][8 rows x 16 B] q boxes and [block][8 rows]
-    // fp16 scale boxes of one packed group each (the tile kernels' maps).
-    // Activation maps: [row][column][16 fp32], one row per box, or all T rows
-    // for the shared expert's segment.
+    // fp16 scale boxes of 1, 2, 4 or 8 consecutive packed groups (the tile
+    // kernels' layout).  Activation maps: [row][column][16 fp32], one row per
+    // box, or all T rows for the shared expert's segment.
     MoeMaps m;
-    const uint64_t gs1 = (uint64_t)kGroupBytesPerBlock * (H / 32);
-    const uint64_t gs2 = (uint64_t)kGroupBytesPerBlock * (I / 32);
     const uint8_t *gu = static_cast<const uint8_t *>(gate_up_experts);
     const uint8_t *dn = static_cast<const uint8_t *>(down_experts);
-    for (int deep = 0; deep < 2; ++deep) {
-        const uint32_t b1 = deep ? kMoeTile1 : 1, b2 = deep ? kMoeTile2 : 1;
-        Q8_CHECK(make_map_3d(deep ? &m.q1r_t : &m.q1r, CU_TENSOR_MAP_DATA_TYPE_UINT8, gu, kColBytes, H / 16,
-                             E * (2 * I / 8), kColBytes, gs1, kColBytes, kMoeCS, b1, true));
-        Q8_CHECK(make_map_3d(deep ? &m.d1r_t : &m.d1r, CU_TENSOR_MAP_DATA_TYPE_UINT16, gu + 256 * (H / 32), 8,
-                             H / 32, E * (2 * I / 8), 16, gs1, 8, kMoeCS / 2, b1, true));
-        Q8_CHECK(make_map_3d(deep ? &m.q2r_t : &m.q2r, CU_TENSOR_MAP_DATA_TYPE_UINT8, dn, kColBytes, I / 16,
-                             E * (H / 8), kColBytes, gs2, kColBytes, kMoeCS, b2, true));
-        Q8_CHECK(make_map_3d(deep ? &m.d2r_t : &m.d2r, CU_TENSOR_MAP_DATA_TYPE_UINT16, dn + 256 * (I / 32), 8,
-                             I / 32, E * (H / 8), 16, gs2, 8, kMoeCS / 2, b2, true));
-    }
+    // weight maps of every box depth (see moe.cuh): [phase][routed|shared][q|scales][depth]
+    auto weight_maps = [&](CUtensorMap(&w)[2][kMoeDepths], const uint8_t *base, int64_t K, int64_t groups)
+        -> q8_status {
+        const uint64_t gs = (uint64_t)kGroupBytesPerBlock * (K / 32);
+        for (int d = 0; d < kMoeDepths; ++d) {
+            Q8_CHECK(make_map_3d(&w[0][d], CU_TENSOR_MAP_DATA_TYPE_UINT8, base, kColBytes, K / 16, groups,
+                                 kColBytes, gs, kColBytes, kMoeCS, 1u << d, true));
+            Q8_CHECK(make_map_3d(&w[1][d], CU_TENSOR_MAP_DATA_TYPE_UINT16, base + 256 * (K / 32), 8, K / 32,
+                                 groups, 16, gs, 8, kMoeCS / 2, 1u << d, true));
+        }
+        return Q8_OK;
+    };
+    Q8_CHECK(weight_maps(m.w[0][0], gu, H, E * (2 * I / 8)));
+    Q8_CHECK(weight_maps(m.w[1][0], dn, I, E * (H / 8)));
     Q8_CHECK(make_map_3d(&m.x1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, H / 16, T, 64, (uint64_t)H * 4, 16, kMoeCS,
                          1, false));
     Q8_CHECK(make_map_3d(&m.x1s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, H / 16, T, 64, (uint64_t)H * 4, 16, kMoeCS,
@@ -760,31 +761,16 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
     Q8_CHECK(make_map_3d(&m.h2r, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.hbuf, 16, I / 16, T * top_k, 64,
                          (uint64_t)I * 4, 16, kMoeCS, 1, false));
     if (has_shared) {
-        const uint64_t gss = (uint64_t)kGroupBytesPerBlock * (Ish / 32);
         const uint8_t *sgu = static_cast<const uint8_t *>(shared_gate_up);
         const uint8_t *sdn = static_cast<const uint8_t *>(shared_down);
-        for (int deep = 0; deep < 2; ++deep) {
-            const uint32_t b1 = deep ? kMoeTile1 : 1, b2 = deep ? kMoeTile2 : 1;
-            Q8_CHECK(make_map_3d(deep ? &m.q1s_t : &m.q1s, CU_TENSOR_MAP_DATA_TYPE_UINT8, sgu, kColBytes, H / 16,
-                                 2 * Ish / 8, kColBytes, gs1, kColBytes, kMoeCS, b1, true));
-            Q8_CHECK(make_map_3d(deep ? &m.d1s_t : &m.d1s, CU_TENSOR_MAP_DATA_TYPE_UINT16, sgu + 256 * (H / 32), 8,
-                                 H / 32, 2 * Ish / 8, 16, gs1, 8, kMoeCS / 2, b1, true));
-            Q8_CHECK(make_map_3d(deep ? &m.q2s_t : &m.q2s, CU_TENSOR_MAP_DATA_TYPE_UINT8, sdn, kColBytes, Ish / 16,
-                                 H / 8, kColBytes, gss, kColBytes, kMoeCS, b2, true));
-            Q8_CHECK(make_map_3d(deep ? &m.d2s_t : &m.d2s, CU_TENSOR_MAP_DATA_TYPE_UINT16, sdn + 256 * (Ish / 32), 8,
-                                 Ish / 32, H / 8, 16, gss, 8, kMoeCS / 2, b2, true));
-        }
+        Q8_CHECK(weight_maps(m.w[0][1], sgu, H, 2 * Ish / 8));
+        Q8_CHECK(weight_maps(m.w[1][1], sdn, Ish, H / 8));
         Q8_CHECK(make_map_3d(&m.h2s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.hsh, 16, Ish / 16, T, 64,
                              (uint64_t)Ish * 4, 16, kMoeCS, (uint32_t)T, false));
     } else {
-        m.q1s = m.q1r;
-        m.d1s = m.d1r;
-        m.q2s = m.q2r;
-        m.d2s = m.d2r;
-        m.q1s_t = m.q1r_t;
-        m.d1s_t = m.d1r_t;
-        m.q2s_t = m.q2r_t;
-        m.d2s_t = m.d2r_t;
+        for (int ph = 0; ph < 2; ++ph)
+            for (int qd = 0; qd < 2; ++qd)
+                for (int d = 0; d < kMoeDepths; ++d) m.w[ph][1][qd][d] = m.w[ph][0][qd][d];
         m.h2s = m.h2r;
     }
     return launch_pdl(moe_kernel_for(nmax_for(T)), dim3((unsigned)dev->sms), dim3(moe_threads(nmax_for(T))), p.smem,
