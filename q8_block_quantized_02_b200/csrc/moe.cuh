@@ -102,6 +102,10 @@ __host__ __device__ constexpr int moe_tg(int phase, int nx) {
     return phase == 1 ? (nx <= 2 ? 6 : nx <= 4 ? 4 : 16 / nx) : (nx <= 4 ? 8 : 32 / nx);
 }
 __host__ __device__ constexpr int moe_halves(int phase) { return phase == 1 ? 2 : 1; }
+// Relative consumer work of an item of a segment with cnt tokens: per 16
+// weights, one dequantisation (~24 instructions) and one dot per token (~10).
+// The routed lists are split over the CTAs by this work, not by item count.
+__host__ __device__ constexpr int moe_item_work(int cnt) { return 24 + 10 * moe_nx(cnt); }
 constexpr int kMoeTile1 = moe_tg(1, 1), kMoeTile2 = moe_tg(2, 1);  // the largest tiles
 // A stage: the weight boxes ([half][item] q boxes, then scale boxes), then
 // one activation box per token.
@@ -133,6 +137,7 @@ struct MoeTable {
     int seg_expert[kMoeMaxSeg];
     int seg_row0[kMoeMaxSeg];          // first pair row
     int seg_cnt[kMoeMaxSeg];           // tokens using it (<= T: picks of a token are distinct)
+    int seg_w0[kMoeMaxSeg + 1];        // work of the segments before it (moe_item_work per item)
     short pair_tok[kMoeMaxPairs];      // pair row -> token
     short pair_slot[kMoeMaxPairs];     // pair row -> slot
     float pair_w[kMoeMaxPairs];        // pair row -> routing weight
@@ -145,6 +150,7 @@ struct MoeTable {
     int pend_n[kMoePend];
     int last_o[kMoePend * kMoeTile2];
     int n_last;                        // groups in last_o whose sums the CTA takes at its end
+    int r0, r1, v0, v1;                // this CTA's routed slices (gate/up, down), set with the table
 };
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
@@ -259,6 +265,30 @@ __device__ __forceinline__ void moe_build_table(MoeTable &tb, const MoeArgs &a, 
     }
     if (lane == 0) tb.n_routed = seg_base;
     __syncwarp();
+    // prefix of the segments' work (<= 128 segments: 4 per lane, then a scan)
+    {
+        int w[4], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int sg = lane * 4 + i;
+            w[i] = sg < seg_base ? moe_item_work(tb.seg_cnt[sg]) : 0;
+            sum += w[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int sg = lane * 4 + i;
+            if (sg <= seg_base) tb.seg_w0[sg] = run;
+            run += w[i];
+        }
+        if (lane == 31) tb.seg_w0[seg_base] = run;  // the total (also when seg_base = 128)
+    }
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         const int p = c * 32 + lane;
@@ -307,6 +337,7 @@ __device__ __forceinline__ void moe_build_table_t1(MoeTable &tb, const MoeArgs &
         rank += ((valid >> j) & 1u) && ej < e;
     }
     if (ok) {
+        tb.seg_w0[rank] = rank * moe_item_work(1);
         tb.seg_expert[rank] = e;
         tb.seg_cnt[rank] = 1;
         tb.seg_row0[rank] = rank;
@@ -317,6 +348,7 @@ __device__ __forceinline__ void moe_build_table_t1(MoeTable &tb, const MoeArgs &
     }
     const int n = __popc(valid);
     if (lane >= n && lane < a.k) tb.tok_order[0][lane] = -1;
+    if (lane == 0) tb.seg_w0[n] = n * moe_item_work(1);
     if (lane == 0) tb.n_routed = n;
     __syncwarp();
 }
@@ -344,21 +376,44 @@ __device__ __forceinline__ MoeRanges moe_ranges_shared(const MoeArgs &a) {
     return rg;
 }
 
-// Each list is split evenly over the CTAs (all of a list's items are equally
-// long), and a CTA walks its slices in list order: shared gate/up (no idx
+// Each list is split over the CTAs (the shared ones evenly, the routed ones
+// by work), and a CTA walks its slices in list order: shared gate/up (no idx
 // needed), routed gate/up, shared down (its h completes first: every CTA
 // starts with the shared gate/up items), routed down.
+// First item of CTA c in a routed list of n items per segment, split by work:
+// the first item starting at or after work position W * c / grid.  Monotone
+// in c, 0 at c = 0 and the item count at c = grid.
+__device__ __forceinline__ int moe_split_routed(const MoeTable &tb, int n, int c, int grid) {
+    // 32-bit throughout: W <= 8192 items x 128 segments x 184 < 2^31, and
+    // W * c / grid = (W / grid) * c + (W % grid) * c / grid exactly
+    const int W = n * tb.seg_w0[tb.n_routed];
+    const int P = (W / grid) * c + (W % grid) * c / grid;
+    if (P >= W) return tb.n_routed * n;
+    int lo = 0, hi = tb.n_routed - 1;  // the segment holding position P
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (n * tb.seg_w0[mid] <= P) lo = mid; else hi = mid - 1;
+    }
+    const int w = tb.seg_w0[lo + 1] - tb.seg_w0[lo];  // one item's work in segment lo
+    const int in = (P - n * tb.seg_w0[lo] + w - 1) / w;
+    return lo * n + (in < n ? in : n);
+}
+
+// The routed slices, computed once (by the table warp, lanes 0-3) into the
+// table; every role then copies them.
+__device__ __forceinline__ void moe_split_routed_all(MoeTable &tb, const MoeArgs &a, int lane) {
+    const int c = blockIdx.x, G = gridDim.x;
+    if (lane == 0) tb.r0 = moe_split_routed(tb, a.I / kGroupRows, c, G);
+    if (lane == 1) tb.r1 = moe_split_routed(tb, a.I / kGroupRows, c + 1, G);
+    if (lane == 2) tb.v0 = moe_split_routed(tb, a.H / kGroupRows, c, G);
+    if (lane == 3) tb.v1 = moe_split_routed(tb, a.H / kGroupRows, c + 1, G);
+    __syncwarp();
+}
 __device__ __forceinline__ void moe_ranges_routed(MoeRanges &rg, const MoeTable &tb, const MoeArgs &a) {
-    const long long G = gridDim.x, c = blockIdx.x;
-    const long long R1 = (long long)tb.n_routed * (a.I / kGroupRows);
-    const long long S2 = (long long)a.nsplit * (a.H / kGroupRows);
-    const long long R2 = (long long)tb.n_routed * (a.H / kGroupRows);
-    rg.r0 = (int)(R1 * c / G);
-    rg.r1 = (int)(R1 * (c + 1) / G);
-    rg.q0 = (int)(S2 * c / G);
-    rg.q1 = (int)(S2 * (c + 1) / G);
-    rg.v0 = (int)(R2 * c / G);
-    rg.v1 = (int)(R2 * (c + 1) / G);
+    rg.r0 = tb.r0;
+    rg.r1 = tb.r1;
+    rg.v0 = tb.v0;
+    rg.v1 = tb.v1;
     rg.table = true;
 }
 
@@ -930,6 +985,7 @@ __global__ void __launch_bounds__(moe_threads(NMAX), 1)
             moe_build_table_t1(tb, a, lane);
         else
             moe_build_table(tb, a, lane);
+        moe_split_routed_all(tb, a, lane);
         if (lane == 0) mbar_arrive(tbl_ready);
         moe_ranges_routed(rg, tb, a);
         const int n_seg = tb.n_routed + a.nsplit;  // phase-2 contributions per output group
