@@ -77,7 +77,7 @@ constexpr uint32_t kMoeQBox = kMoeCS * kColBytes;  // one item's q box
 constexpr uint32_t kMoeDBox = kMoeCS * 8;          // one item's scale box ([CS/2][8] fp16)
 constexpr uint32_t kMoeXRow = kMoeCS * 64;         // one token's activation box
 constexpr int kMoeMaxStages = 8;
-constexpr int kMoeRedBufs = 4;                 // partial-sum buffers between consumers and the epilogue warp
+constexpr int kMoeRedBufs = 3;                 // partial-sum buffers between consumers and the epilogue warp
 constexpr int kMoeBarBytes = 256;              // mbarriers: full, empty (<= 8 each), red full/free (4 each), table
 constexpr int kMoeRedMax = 64;                 // partial-sum slots per column quad and tile
 constexpr int kMoePend = 32;                   // phase-2 tiles the epilogue warp counts at once
@@ -143,15 +143,18 @@ struct MoeTable {
     float pair_w[kMoeMaxPairs];        // pair row -> routing weight
     signed char tok_order[kMoeMaxT][kMoeMaxK];  // token's slots by ascending expert id, -1 after
     int pick[kMoeMaxPairs];            // idx, -1 where the pick was rejected
-    int counts[kMoeMaxE];              // per-expert pick count, then expert -> segment
-    // epilogue warp: phase-2 tiles stored but not yet counted (first group,
-    // groups), and the output groups whose sums it takes
+    union {
+        int counts[kMoeMaxE];          // while building: per-expert pick count, then expert -> segment
+        int last_o[kMoePend * kMoeTile2];  // at the end: output groups whose sums this CTA takes
+    };
+    // epilogue warp: phase-2 tiles stored but not yet counted (first group, groups)
     int pend_o0[kMoePend];
     int pend_n[kMoePend];
-    int last_o[kMoePend * kMoeTile2];
     int n_last;                        // groups in last_o whose sums the CTA takes at its end
     int r0, r1, v0, v1;                // this CTA's routed slices (gate/up, down), set with the table
 };
+
+static_assert(kMoeMaxE == kMoePend * kMoeTile2, "the table's counts and last_o share storage");
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
     unsigned v;
