@@ -44,6 +44,24 @@ WORKLOAD = ("qwen2.5-0.5b batch-1 decode matmul set: 24 x {qkv 1152x896, wo 896x
             "gate_up 9728x896 + SwiGLU, down 896x4864} + lm_head 151936x896, Q8_0 weights, fp32 x")
 
 
+def max_over_ranks(value, world, device):
+    """The largest `value` over the job's ranks, received by every rank: a
+    job's time is its slowest rank's.  `value` itself with one rank."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world, units_per_rank, elapsed_max):
+    """Whole-job throughput of `world` independent replicas: the units all
+    ranks processed over the slowest rank's time."""
+    return world * units_per_rank / elapsed_max
+
+
 def measured_hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -279,11 +297,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    elapsed = t_start.elapsed_time(t_end) / 1e3
-    if world > 1:
-        t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(t_start.elapsed_time(t_end) / 1e3, world, dev)
 
     # ---- per-kernel launch duration: each class's chain replayed on its own ----
     reps = max(10, min(100, args.steps // 20))
@@ -320,11 +334,7 @@ def run_ours(args):
         stream.synchronize()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_elapsed = e0.elapsed_time(e1) / 1e3
-    if world > 1:
-        t = torch.tensor([e2e_elapsed], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_elapsed = float(t.item())
+    e2e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
 
     # ---- CPU oracle baseline (rank 0, single GPU only) ----
     cpu = None
@@ -344,7 +354,7 @@ def run_ours(args):
         return 0
 
     peak, peak_kind = measured_hbm_peak()
-    tok_s = world * args.steps / elapsed
+    tok_s = replica_throughput(world, args.steps, elapsed)
     gbs = step_bytes * args.steps / elapsed / 1e9  # per GPU
     dom = kstats["q8_gemv_n1"]
     achieved = dom["GBps"]
@@ -392,7 +402,7 @@ def run_ours(args):
                            "bytes_per_launch": int(k["bytes_per_launch"]),
                            "GBps": round(k["GBps"], 1)} for name, k in kstats.items()},
         "e2e": {
-            "value": round(world * e2e_steps / e2e_elapsed, 2),
+            "value": round(replica_throughput(world, e2e_steps, e2e_elapsed), 2),
             "unit": "tok/s",
             "h2d_bytes_per_step": int(x_total * 4),
             "d2h_bytes_per_step": int(y_bufs[lm].numel() * 4),
