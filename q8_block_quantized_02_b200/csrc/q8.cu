@@ -118,9 +118,11 @@ static TilePlan plan_tile(int64_t units, int64_t C, int64_t N, int mode, int sms
     const bool cols_path = nb <= 4;  // column-owner kernel (see tile_gemm.cuh)
     const int64_t grid = units < sms ? units : sms;
     const int64_t upc = ceil_div(units, grid);
-    // many tiles per CTA: take the 16-warp kernel (it fills the SM on its own);
-    // otherwise stay within half an SM so the next kernel can co-reside
-    const bool wide = nb == 1 && upc >= 32;
+    // much work per CTA (many row groups, or few very long ones): take the
+    // 16-warp kernel (it fills the SM on its own); otherwise stay within half
+    // an SM so the next kernel can co-reside
+    const int64_t cta_bytes = upc * (swiglu ? 2 : 1) * C * (kColBytes + 8);
+    const bool wide = nb == 1 && (upc >= 32 || cta_bytes >= 256 * 1024);
     const KernelShape ks = kernel_shape(nb, mode, wide);
     int64_t tg = cols_path ? ks.tgm : std::min<int64_t>(swiglu ? 8 : 16, pow2_ceil(upc));
     tg = std::min<int64_t>(tg, upc);  // a stage never holds more units than a CTA owns
