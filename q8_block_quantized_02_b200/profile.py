@@ -3,6 +3,7 @@
     python -m q8_block_quantized_02_b200.profile --op gemv --M 151936 --K 896 --N 1
     python -m q8_block_quantized_02_b200.profile --op q8q8 --M 37888 --K 3584 --N 16
     python -m q8_block_quantized_02_b200.profile --op moe --T 1
+    python -m q8_block_quantized_02_b200.profile --op readpeak
 
 Weights follow the synthetic Q8_0 recipe (q uniform in [-127, 127], d =
 |N(0,1)| * 0.02) and activations are N(0,1).  Enough packed copies of the
@@ -24,6 +25,11 @@ are routed up front (q8_moe_route, not timed) and the timed calls cycle
 through them, so consecutive calls select different experts.  Bytes per
 call count each call's distinct selected experts plus the shared expert once
 (34 B per 32 weights).
+
+`--op readpeak` is a reference figure, not a libq8 product: the HBM read rate
+of a plain reduction (torch.sum over 4 GiB of fp32, so every byte is read
+once and nothing is written back), the read-only counterpart of the measured
+copy peak.
 """
 from __future__ import annotations
 
@@ -39,7 +45,7 @@ if ROOT not in sys.path:
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--op", choices=["gemv", "swiglu", "q8q8", "moe"], default="gemv",
+    ap.add_argument("--op", choices=["gemv", "swiglu", "q8q8", "moe", "readpeak"], default="gemv",
                     help="q8_gemv, q8_gate_up_swiglu (M = rows of the stacked gate|up matrix) "
                          "or q8_quantize_act + q8q8_gemv (only q8q8_gemv is timed)")
     ap.add_argument("--M", type=int, default=151936)
@@ -59,6 +65,8 @@ def main(argv=None) -> int:
     args = ap.parse_args(argv)
     if args.op == "moe":
         return _moe(args)
+    if args.op == "readpeak":
+        return _readpeak(args)
 
     import numpy as np
     import torch
@@ -120,6 +128,31 @@ def main(argv=None) -> int:
                       "weight_GBps": round(weight_bytes / (us * 1e-6) / 1e9, 1), "copies": copies,
                       "reps": args.reps, "device_error": word}), flush=True)
     return 0 if st == 0 else 1
+
+
+def _readpeak(args) -> int:
+    import torch
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    n = (4 << 30) // 4
+    a = torch.ones(n, dtype=torch.float32, device=dev)
+    out = torch.empty((), dtype=torch.float32, device=dev)
+    for _ in range(max(3, args.warmup)):
+        torch.sum(a, 0, out=out)
+    torch.cuda.synchronize()
+    reps = max(5, min(args.reps, 50))
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(reps):
+        torch.sum(a, 0, out=out)
+    t1.record()
+    torch.cuda.synchronize()
+    us = t0.elapsed_time(t1) * 1e3 / reps
+    assert abs(float(out.item()) - n) <= 1e-3 * n
+    print(json.dumps({"op": "readpeak", "bytes": n * 4, "us_per_call": round(us, 2),
+                      "read_GBps": round(n * 4 / (us * 1e-6) / 1e9, 1), "reps": reps}), flush=True)
+    return 0
 
 
 def _moe(args) -> int:
