@@ -21,17 +21,19 @@ namespace q8 {
 using TileKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
                            TileArgs);
 
-// `wide` selects the 16-consumer-warp column kernel (N = 1 only): more warps
-// per SM for matrices with many tiles per CTA; the 8-warp kernels leave room
-// for the next kernel on the stream to become resident early.
+// `wide` selects, at N = 1, the 16-consumer-warp column kernel (more warps
+// per SM for matrices with much work per CTA; the 8-warp kernels leave room
+// for the next kernel on the stream to become resident early), and for N > 4
+// the group-owner build that runs two CTAs per SM.
 template <int MODE>
 static TileKernel tile_kernel_mode(int nmax, bool wide) {
     switch (nmax) {
         case 1: return wide ? &cols_kernel<1, MODE, 16> : &cols_kernel<1, MODE, 8>;
         case 2: return &cols_kernel<2, MODE, 8>;
         case 4: return &cols_kernel<4, MODE, 8>;
-        case 8: return &tile_gemm_kernel<8, MODE>;
-        default: return &tile_gemm_kernel<16, MODE>;
+        case 8: return wide ? &tile_gemm_kernel<8, MODE, 2> : &tile_gemm_kernel<8, MODE, 1>;
+        default:
+            return wide && tile_two_ctas_ok(16, MODE) ? &tile_gemm_kernel<16, MODE, 2> : &tile_gemm_kernel<16, MODE, 1>;
     }
 }
 
@@ -75,10 +77,10 @@ static KernelShape kernel_shape(int nmax, int mode, bool wide = false) {
 
 static cudaError_t setup_tile_kernels(int max_smem) {
     const int nm[5] = {1, 2, 4, 8, 16};
-    for (int i = 0; i < 6; ++i)
+    for (int i = 0; i < 8; ++i)
         for (int mode = 0; mode < 3; ++mode) {
             const void *k = reinterpret_cast<const void *>(
-                i < 5 ? tile_kernel_for(nm[i], mode) : tile_kernel_for(1, mode, true));
+                i < 5 ? tile_kernel_for(nm[i], mode) : tile_kernel_for(i == 5 ? 1 : i == 6 ? 8 : 16, mode, true));
             cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
             if (e != cudaSuccess) return e;
             // every tile kernel asks for the largest shared-memory carveout, so
@@ -116,13 +118,18 @@ static TilePlan plan_tile(int64_t units, int64_t C, int64_t N, int mode, int sms
     const bool swiglu = mode == kModeSwiGLU;
     const int nb = nmax_for(N);
     const bool cols_path = nb <= 4;  // column-owner kernel (see tile_gemm.cuh)
-    const int64_t grid = units < sms ? units : sms;
+    // the group-owner kernel (N > 4) is bound by its FP32 issue: two CTAs per
+    // SM (each within half of it) double the warps that hide the FMA latency,
+    // when there are units enough for whole tiles of 8 per CTA
+    const bool dual = !cols_path && tile_two_ctas_ok(nb, mode) && units >= 16 * sms;
+    const int64_t ctas = dual ? 2 * sms : sms;
+    const int64_t grid = units < ctas ? units : ctas;
     const int64_t upc = ceil_div(units, grid);
     // much work per CTA (many row groups, or few very long ones): take the
     // 16-warp kernel (it fills the SM on its own); otherwise stay within half
     // an SM so the next kernel can co-reside
     const int64_t cta_bytes = upc * (swiglu ? 2 : 1) * C * (kColBytes + 8);
-    const bool wide = nb == 1 && (upc >= 32 || cta_bytes >= 256 * 1024);
+    const bool wide = (nb == 1 && (upc >= 32 || cta_bytes >= 256 * 1024)) || dual;
     const KernelShape ks = kernel_shape(nb, mode, wide);
     int64_t tg = cols_path ? ks.tgm : std::min<int64_t>(swiglu ? 8 : 16, pow2_ceil(upc));
     tg = std::min<int64_t>(tg, upc);  // a stage never holds more units than a CTA owns

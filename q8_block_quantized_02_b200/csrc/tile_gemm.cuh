@@ -844,8 +844,17 @@ __device__ __forceinline__ void consume_groups(uint8_t *smem, uint32_t full0, ui
     }
 }
 
-template <int NMAX, int MODE>
-__global__ void __launch_bounds__(kTileThreads, 1)
+// The group-owner kernel comes in two builds: one CTA per SM (no register
+// limit but the SM's), and CTAS = 2, two CTAs per SM, each within half of it
+// (96 registers a thread): twice the warps to hide the FMA latency when a
+// matrix has row groups enough to fill both.  SwiGLU at 16 columns keeps one
+// (its gate and up accumulators need the registers).
+__host__ __device__ constexpr bool tile_two_ctas_ok(int nmax, int mode) {
+    return !(mode == kModeSwiGLU && nmax == 16);
+}
+
+template <int NMAX, int MODE, int CTAS>
+__global__ void __launch_bounds__(kTileThreads, CTAS)
     tile_gemm_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap td,
                      const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap td1,
                      const __grid_constant__ CUtensorMap tx, const TileArgs a) {
