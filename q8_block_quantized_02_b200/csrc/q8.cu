@@ -9,6 +9,7 @@
 #include "pack.cuh"
 #include "q8q8.cuh"
 #include "q8q8_mma.cuh"
+#include "f32_mma.cuh"
 #include "route.cuh"
 #include "tile_gemm.cuh"
 #include "moe.cuh"
@@ -294,9 +295,19 @@ static q8_status run_resident(const TilePlan &plan, const void *W, const float *
                       swiglu ? "q8_gate_up_swiglu launch" : "q8_gemv launch", tq, td, x, a);
 }
 
+static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_out, int64_t K,
+                        int64_t N, bool swiglu, cudaStream_t stream);
+
+#ifndef Q8_FM_MIN_N
+#define Q8_FM_MIN_N 5
+#endif
+constexpr int64_t kFmMinN = Q8_FM_MIN_N;  // smallest N of fp32 activations sent to the tensor cores
+
 static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, float *y,
                           int64_t rows_out, int64_t K, int64_t N, int mode, cudaStream_t stream) {
     const bool swiglu = mode == kModeSwiGLU;
+    if (mode != kModeQ8Q8 && N >= kFmMinN)
+        return run_fm(W, static_cast<const float *>(x), y, rows_out, K, N, swiglu, stream);
     const DeviceInfo *dev = nullptr;
     Q8_CHECK(device_info(&dev));
     const int64_t B = K / 32, C = K / 16;
@@ -418,6 +429,91 @@ static q8_status run_mma(const void *W, const int8_t *xq, const uint16_t *xd, fl
                          kMmaN, kMmaCS, false));
     return launch_pdl_cluster(q8q8_mma_kernel, dim3(p.grid), dim3(kMmaThreads), p.smem, stream,
                               "q8q8_gemv (tensor cores) launch", (unsigned)p.a.split, tq, td, tx, p.a);
+}
+
+// ---------------------------------------------------------------------------
+// fp32 activations on the tensor cores (S3 / S4, 5..16 activation columns)
+// ---------------------------------------------------------------------------
+static cudaError_t setup_fm_kernels(int max_smem) {
+    const void *ks[4] = {reinterpret_cast<const void *>(&f32_mma_kernel<false, 4>),
+                         reinterpret_cast<const void *>(&f32_mma_kernel<false, 8>),
+                         reinterpret_cast<const void *>(&f32_mma_kernel<true, 4>),
+                         reinterpret_cast<const void *>(&f32_mma_kernel<true, 8>)};
+    for (const void *k : ks) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+static RegisterSetup g_reg_fm(setup_fm_kernels);
+
+struct FmPlan {
+    FmArgs a;
+    int grid;  // CTAs (a multiple of a.split)
+    size_t smem;
+};
+
+// One CTA per SM.  A tile is 128 output rows (SwiGLU: 64 outputs, their gate
+// and up rows).  With at least as many tiles as SMs each cluster is one CTA
+// walking a contiguous tile range; with fewer, every tile gets a cluster of up
+// to 8 CTAs that split K between them.
+static FmPlan plan_fm(int64_t rows_out, int64_t K, int64_t N, bool swiglu, int sms) {
+    FmPlan p;
+    FmArgs &a = p.a;
+    a = FmArgs{};
+    const int64_t B = K / 32;
+    const int64_t tiles = ceil_div(rows_out, swiglu ? 64 : 128);
+    int64_t split = 1, clusters = sms;
+    if (tiles < sms) {
+        split = std::min<int64_t>(kFmMaxSplit, sms / tiles);
+        split = std::min<int64_t>(split, B);  // every CTA keeps at least one block
+        if (split < 1) split = 1;
+        clusters = tiles;
+    }
+    const int64_t blocks = ceil_div(B, split);
+    const int64_t per_cta = ceil_div(tiles, clusters) * ceil_div(blocks, kFmSB);
+    a.M_out = (int)rows_out;
+    a.N = (int)N;
+    a.B = (int)B;
+    a.tiles = (int)tiles;
+    a.split = (int)split;
+    a.stages = (int)std::max<int64_t>(1, std::min<int64_t>(kFmMaxStages, per_cta));
+    a.up_group0 = swiglu ? (int)(rows_out / kGroupRows) : 0;
+    p.grid = (int)(clusters * split);
+    p.smem = fm_smem_bytes(a.stages);
+    return p;
+}
+
+static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_out, int64_t K,
+                        int64_t N, bool swiglu, cudaStream_t stream) {
+    const DeviceInfo *dev = nullptr;
+    Q8_CHECK(device_info(&dev));
+    const int64_t B = K / 32, C = K / 16;
+    const int64_t units = ceil_div(rows_out, kGroupRows);
+    const int64_t groups = swiglu ? 2 * units : units;
+    FmPlan p = plan_fm(rows_out, K, N, swiglu, dev->sms);
+    if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
+    p.a.y = y;
+    const uint64_t gstride = (uint64_t)kGroupBytesPerBlock * B;
+    const uint8_t *dbase = static_cast<const uint8_t *>(W) + 256 * B;
+    CUtensorMap tq, td;
+    // weights: [group][16-byte column][8 rows x 16 B], 8 groups x kFmCS columns a box
+    Q8_CHECK(make_map_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, kColBytes, C, groups, kColBytes,
+                         gstride, kColBytes, kFmCS, 8, true));
+    // scales: [group][block][8 rows] fp16, 8 groups x kFmSB blocks a box
+    Q8_CHECK(make_map_3d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT16, dbase, 8, B, groups, 16, gstride, 8,
+                         kFmSB, 8, true));
+    // the activations are read by the kernel's splitter warps with plain loads;
+    // each epilogue warp takes 4 activation rows up to N = 8, else 8
+    using FmKernel = void (*)(CUtensorMap, CUtensorMap, const float *, FmArgs);
+    const FmKernel k = swiglu ? (N <= 8 ? &f32_mma_kernel<true, 4> : &f32_mma_kernel<true, 8>)
+                              : (N <= 8 ? &f32_mma_kernel<false, 4> : &f32_mma_kernel<false, 8>);
+    return launch_pdl_cluster(k, dim3(p.grid), dim3(kFmThreads), p.smem, stream,
+                              swiglu ? "q8_gate_up_swiglu (tensor cores) launch" : "q8_gemv (tensor cores) launch",
+                              (unsigned)p.a.split, tq, td, x, p.a);
 }
 
 // ---------------------------------------------------------------------------
