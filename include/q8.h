@@ -122,7 +122,14 @@ q8_status q8_unpack_weights(const void *packed, int64_t M, int64_t K, void *gguf
  * overwritten.  fp32 arithmetic; each output is within 1e-5 * sum_k |w x| of
  * the exact value.  The Q8 N=1 decode product of "Lumen v0.3.0" (Phase 7.G)
  * and the "skuznetsov/cogni-ml" cuda_q8_gemv_probe ("Build Qwen CLIs"),
- * extended to N <= 16 columns.  N > 16 -> Q8_ERR_UNSUPPORTED. */
+ * extended to N <= 16 columns.  N > 16 -> Q8_ERR_UNSUPPORTED.
+ * N <= 4: fp32 dequantise-and-FMA on the CUDA cores.  5 <= N <= 16: the
+ * tensor cores (tcgen05.mma kind::i8, one MMA per Q8_0 block) take the packed
+ * int8 q against an exact three-term int8 split of each 32-block of x,
+ * x = s (q0 + q1/254 + q2/254^2) with a power-of-two s per block (residual
+ * below 2.5e-7 of the block's max |x|), and an fp32 epilogue applies d and s
+ * per block; the same 1e-5 bound holds.  Activation blocks whose max |x| is
+ * below 2^-121 lose relative accuracy there; non-finite x is undefined. */
 q8_status q8_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
                   q8_stream_t stream);
 
@@ -136,7 +143,8 @@ q8_status q8_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K,
  * projections of the "skuznetsov/cogni-ml" FFN probe, "Build Qwen CLIs"; the
  * SwiGLU MLP of the "augur" README, "Features").  I must be a multiple of 8.
  * x: [N][K] fp32.  h: [N][I] fp32, fully overwritten.  One launch; g and u
- * never leave the chip. */
+ * never leave the chip.  5 <= N <= 16 runs on the tensor cores as q8_gemv
+ * does (a tile holds 64 gate rows and their 64 up rows). */
 q8_status q8_gate_up_swiglu(const void *W, const float *x, float *h, int64_t I, int64_t K,
                             int64_t N, q8_stream_t stream);
 
@@ -212,10 +220,9 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
 /* Same product as q8_moe_gemv, without a workspace argument.  The pages have
  * no counterpart: this variant exists for callers that cannot allocate device
  * memory when they call -- for example a plug-in that is handed finished
- * device buffers by a host framework owning the memory pool, code that runs
- * while a stream is being captured into a CUDA graph (allocation calls are
- * not permitted there), or a decode loop that must not risk an allocation's
- * implicit synchronisation.
+ * device buffers by a host framework that owns the memory pool and gives it
+ * no allocator, or a decode loop that must not risk an allocation's implicit
+ * synchronisation in the middle of a token.
  * Scratch comes from a fixed 4 MiB array in the library's device memory, held
  * by every GPU that loads the library until the process exits.  Sizes whose
  * q8_moe_workspace_bytes() exceeds 4 MiB are rejected with
@@ -223,12 +230,11 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
  * allocated or freed.
  * The first call on each device looks up the array's device address (with
  * that device current); make that first call before any stream capture.
- * All calls share the one array.  It starts zero-filled and every call that
- * completes without a device error leaves it ready for the next; after a
- * device error the next no-alloc call may compute wrong values, so a process
- * should treat that error as fatal.  Calls that may run at the same time on the GPU
- * (different streams without an ordering between them) race on the array and
- * must not be issued. */
+ * All calls share the one array, which keeps the last call's contents: each
+ * call first clears the array's counter region on `stream`
+ * (cudaMemsetAsync), then runs the MoE kernel.  Calls that may run at the
+ * same time on the GPU (different streams without an ordering between them)
+ * race on the array and must not be issued. */
 q8_status q8_moe_gemv_noalloc(const void *gate_up_experts, const void *down_experts,
                               const void *shared_gate_up, const void *shared_down,
                               const int32_t *idx, const float *w, const float *x, float *y,

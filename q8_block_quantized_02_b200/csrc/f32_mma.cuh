@@ -55,10 +55,10 @@
 // activation buffers, running ahead of the MMAs.  Warps: 0 issues TMA (weight
 // boxes of the first stages before griddepcontrol.wait), 1 owns tensor memory
 // and issues the MMAs, 2..9 split (warp 2 + i takes activation rows i and
-// i + 8), 10..17 are the epilogue: warp w reads TMEM lanes 32 * (w % 4) .. and
-// TOK activation rows from TOK * ((w - 10) / 4) (TOK = 4 for N <= 8, else 8),
-// so every epilogue warp has work at any N, and no epilogue warp waits for a
-// split.  With fewer 128-row tiles than
+// i + 8), 10..25 are the epilogue: warp w reads TMEM lanes 32 * (w % 4) .. and
+// TOK activation rows from TOK * ((w - 10) / 4) (TOK = 2 for N <= 8, else 4),
+// so the epilogue's work spreads over 16 warps at any N, and no epilogue warp
+// waits for a split.  With fewer 128-row tiles than
 // SMs, K is split over a cluster of up to 8 CTAs and the partial sums meet in
 // the leader in rank order (bit-identical results from run to run).
 // Every wait is bounded; a stalled pipeline records an error, waits for its
@@ -79,7 +79,7 @@ constexpr int kFmHalves = kFmSB / kFmHalfBlocks;  // 2
 constexpr uint32_t kFmBlockCols = 64;             // TMEM columns per block (48 used)
 constexpr uint32_t kFmTmemCols = kFmSB * kFmBlockCols;  // 512
 constexpr int kFmSplitWarps = 8;
-constexpr int kFmEpiWarps = 8;
+constexpr int kFmEpiWarps = 16;
 constexpr int kFmEpiThreads = kFmEpiWarps * 32;
 constexpr int kFmThreads = 64 + 32 * kFmSplitWarps + kFmEpiThreads;  // producer, MMA, splitters, epilogue
 constexpr int kFmNB = 3;                          // activation buffers (pieces + table)
@@ -132,21 +132,19 @@ __device__ __forceinline__ void tmem_ld4_async(uint32_t taddr, uint32_t *v) {
                  : "r"(taddr)
                  : "memory");
 }
-__device__ __forceinline__ void tmem_ld8_cols(uint32_t taddr, uint32_t *v) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                   "=r"(v[7])
+__device__ __forceinline__ void tmem_ld2_async(uint32_t taddr, uint32_t *v) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];"
+                 : "=r"(v[0]), "=r"(v[1])
                  : "r"(taddr)
                  : "memory");
 }
-// Waits for every earlier tcgen05.ld of the thread; names 16 of the loaded
+// Waits for every earlier tcgen05.ld of the thread; names 8 of the loaded
 // registers so that no use of them is scheduled before it (called once per
-// 16 registers: the later calls return at once).
-__device__ __forceinline__ void tmem_wait_ld16(uint32_t *v) {
+// 8 registers: the later calls return at once).
+__device__ __forceinline__ void tmem_wait_ld8(uint32_t *v) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]),
-                   "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]),
-                   "+r"(v[14]), "+r"(v[15])
+                   "+r"(v[7])
                  :
                  : "memory");
 }
@@ -246,40 +244,33 @@ __device__ __forceinline__ void fm_split_row(uint8_t *ab, const uint4 (&xr)[2], 
 // three TMEM dots in v and (s, corrections) from the activation buffer's
 // table.  FULL: every block of the batch is inside the K range.
 template <bool FULL, int TOK, int LB>
-__device__ __forceinline__ void fm_epilogue_blocks(uint64_t (&acc2)[TOK / 2], const uint32_t (&v)[LB][kFmPieces][TOK],
+__device__ __forceinline__ void fm_epilogue_blocks(float (&acc)[TOK], const uint32_t (&v)[LB][kFmPieces][TOK],
                                                    int jb, int nb, const uint8_t *st, const uint8_t *ab, int g, int r,
                                                    int n0) {
-    const uint32_t un = __float_as_uint(-12582912.0f);
-    const uint64_t nm2 = pack_u32x2(un, un);
-    const uint32_t c1 = __float_as_uint(1.0f / 254.0f), c2 = __float_as_uint(1.0f / 64516.0f);
-    const uint64_t c1x2 = pack_u32x2(c1, c1), c2x2 = pack_u32x2(c2, c2);
 #pragma unroll
     for (int jj = 0; jj < LB; ++jj) {
         const int j = jb + jj;
         if (!FULL && j >= nb) break;
         const float dw = __half2float(*reinterpret_cast<const __half *>(st + kFmDOff + (g * kFmSB + j) * 16 + r * 2));
-        const uint64_t dw2 = pack_u32x2(__float_as_uint(dw), __float_as_uint(dw));
         const uint4 *tab = reinterpret_cast<const uint4 *>(ab + kFmTabOff + (j * kFmN + n0) * 16);
 #pragma unroll
-        for (int p = 0; p < TOK / 2; ++p) {
-            const uint4 e0 = tab[2 * p], e1 = tab[2 * p + 1];
-            const uint64_t f0 = add_f32x2(pack_u32x2(v[jj][0][2 * p] + e0.y, v[jj][0][2 * p + 1] + e1.y), nm2);
-            const uint64_t f1 = add_f32x2(pack_u32x2(v[jj][1][2 * p] + e0.z, v[jj][1][2 * p + 1] + e1.z), nm2);
-            const uint64_t f2 = add_f32x2(pack_u32x2(v[jj][2][2 * p] + e0.w, v[jj][2][2 * p + 1] + e1.w), nm2);
-            uint64_t c = fma_f32x2(f1, c1x2, f0);
-            c = fma_f32x2(f2, c2x2, c);
-            const uint64_t sc = mul_f32x2(dw2, pack_u32x2(e0.x, e1.x));
-            acc2[p] = fma_f32x2(c, sc, acc2[p]);
+        for (int t = 0; t < TOK; ++t) {
+            const uint4 e = tab[t];
+            const float f0 = __uint_as_float(v[jj][0][t] + e.y) - 12582912.0f;
+            const float f1 = __uint_as_float(v[jj][1][t] + e.z) - 12582912.0f;
+            const float f2 = __uint_as_float(v[jj][2][t] + e.w) - 12582912.0f;
+            const float c = fmaf(f2, 1.0f / 64516.0f, fmaf(f1, 1.0f / 254.0f, f0));
+            acc[t] = fmaf(c, dw * __uint_as_float(e.x), acc[t]);
         }
     }
 }
 
-// TOK: activation rows per epilogue warp (4 for N <= 8, else 8).
+// TOK: activation rows per epilogue warp (2 for N <= 8, else 4).
 template <bool SWIGLU, int TOK>
 __global__ void __launch_bounds__(kFmThreads, 1)
     f32_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap td,
                    const float *__restrict__ x, const FmArgs a) {
-    constexpr int LB = 16 / TOK;  // blocks per TMEM load batch (48 registers)
+    constexpr int LB = 8 / TOK;  // blocks per TMEM load batch (24 registers)
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = a.split;
@@ -455,7 +446,7 @@ __global__ void __launch_bounds__(kFmThreads, 1)
         }
     } else {
         // ------------------------------ epilogue ------------------------------
-        const int ew = warp - 2 - kFmSplitWarps;  // epilogue warp 0..7
+        const int ew = warp - 2 - kFmSplitWarps;  // epilogue warp 0..15
         const int q = warp & 3;                   // TMEM lane quarter of this warp
         const int n0 = TOK * (ew >> 2);           // its activation rows n0 .. n0 + TOK - 1
         const bool active = n0 < a.N;
@@ -463,11 +454,11 @@ __global__ void __launch_bounds__(kFmThreads, 1)
         const int g = row >> 3, r = row & 7;      // packed group (0..15) and row in it
         const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + n0;
         pdl_wait_and_trigger();  // the outputs belong to the previous grid until now
-        uint64_t acc2[TOK / 2];  // fp32 pairs (n0 + 2p, n0 + 2p + 1)
+        float acc[TOK];
         int it = 0;
         for (int tl = 0; tl < n_tiles; ++tl) {
 #pragma unroll
-            for (int p = 0; p < TOK / 2; ++p) acc2[p] = 0ull;
+            for (int t = 0; t < TOK; ++t) acc[t] = 0.f;
             for (int ks = 0; ks < ksteps; ++ks, ++it) {
                 const int slot = it % a.stages, ab = it % kFmNB;
                 const uint8_t *st = smem + (size_t)slot * kFmStageBytes;
@@ -491,15 +482,15 @@ __global__ void __launch_bounds__(kFmThreads, 1)
 #pragma unroll
                                 for (int k = 0; k < kFmPieces; ++k) {
                                     const uint32_t ta = taddr + (jb + jj) * kFmBlockCols + k * kFmN;
-                                    if (TOK == 8)
-                                        tmem_ld8_cols(ta, v[jj][k]);
-                                    else
+                                    if (TOK == 4)
                                         tmem_ld4_async(ta, v[jj][k]);
+                                    else
+                                        tmem_ld2_async(ta, v[jj][k]);
                                 }
                             uint32_t *vf = &v[0][0][0];
-                            tmem_wait_ld16(vf);
-                            tmem_wait_ld16(vf + 16);
-                            tmem_wait_ld16(vf + 32);
+                            tmem_wait_ld8(vf);
+                            tmem_wait_ld8(vf + 8);
+                            tmem_wait_ld8(vf + 16);
                         }
                         if (bt == kFmHalfBlocks / LB - 1) {
                             // every load of this half is done: the MMAs may refill it
@@ -509,9 +500,9 @@ __global__ void __launch_bounds__(kFmThreads, 1)
                         }
                         if (work) {
                             if (nb == kFmSB)
-                                fm_epilogue_blocks<true, TOK, LB>(acc2, v, jb, nb, st, abuf, g, r, n0);
+                                fm_epilogue_blocks<true, TOK, LB>(acc, v, jb, nb, st, abuf, g, r, n0);
                             else
-                                fm_epilogue_blocks<false, TOK, LB>(acc2, v, jb, nb, st, abuf, g, r, n0);
+                                fm_epilogue_blocks<false, TOK, LB>(acc, v, jb, nb, st, abuf, g, r, n0);
                         }
                     }
                     if (!okh) break;
@@ -523,13 +514,7 @@ __global__ void __launch_bounds__(kFmThreads, 1)
                 }
             }
             // ---- tile done: K-split partials meet in the leader, rank order ----
-            float acc[TOK];
-#pragma unroll
-            for (int p = 0; p < TOK / 2; ++p) {
-                const float2 f = unpack_f32x2(acc2[p]);
-                acc[2 * p] = f.x;
-                acc[2 * p + 1] = f.y;
-            }
+
             bool store = true;
             if (S > 1) {
                 if (rank != 0) {

@@ -435,10 +435,10 @@ static q8_status run_mma(const void *W, const int8_t *xq, const uint16_t *xd, fl
 // fp32 activations on the tensor cores (S3 / S4, 5..16 activation columns)
 // ---------------------------------------------------------------------------
 static cudaError_t setup_fm_kernels(int max_smem) {
-    const void *ks[4] = {reinterpret_cast<const void *>(&f32_mma_kernel<false, 4>),
-                         reinterpret_cast<const void *>(&f32_mma_kernel<false, 8>),
-                         reinterpret_cast<const void *>(&f32_mma_kernel<true, 4>),
-                         reinterpret_cast<const void *>(&f32_mma_kernel<true, 8>)};
+    const void *ks[4] = {reinterpret_cast<const void *>(&f32_mma_kernel<false, 2>),
+                         reinterpret_cast<const void *>(&f32_mma_kernel<false, 4>),
+                         reinterpret_cast<const void *>(&f32_mma_kernel<true, 2>),
+                         reinterpret_cast<const void *>(&f32_mma_kernel<true, 4>)};
     for (const void *k : ks) {
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
         if (e != cudaSuccess) return e;
@@ -507,10 +507,10 @@ static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_ou
     Q8_CHECK(make_map_3d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT16, dbase, 8, B, groups, 16, gstride, 8,
                          kFmSB, 8, true));
     // the activations are read by the kernel's splitter warps with plain loads;
-    // each epilogue warp takes 4 activation rows up to N = 8, else 8
+    // each epilogue warp takes 2 activation rows up to N = 8, else 4
     using FmKernel = void (*)(CUtensorMap, CUtensorMap, const float *, FmArgs);
-    const FmKernel k = swiglu ? (N <= 8 ? &f32_mma_kernel<true, 4> : &f32_mma_kernel<true, 8>)
-                              : (N <= 8 ? &f32_mma_kernel<false, 4> : &f32_mma_kernel<false, 8>);
+    const FmKernel k = swiglu ? (N <= 8 ? &f32_mma_kernel<true, 2> : &f32_mma_kernel<true, 4>)
+                              : (N <= 8 ? &f32_mma_kernel<false, 2> : &f32_mma_kernel<false, 4>);
     return launch_pdl_cluster(k, dim3(p.grid), dim3(kFmThreads), p.smem, stream,
                               swiglu ? "q8_gate_up_swiglu (tensor cores) launch" : "q8_gemv (tensor cores) launch",
                               (unsigned)p.a.split, tq, td, x, p.a);
@@ -898,8 +898,10 @@ q8_status q8_moe_gemv_noalloc(const void *gate_up_experts, const void *down_expe
     }
     void *scratch = nullptr;
     Q8_CHECK(moe_noalloc_scratch(&scratch));
-    // The array starts zero-filled (a static device array) and every call
-    // leaves its counters zero again, as the MoE kernel requires.
+    // The array keeps whatever the previous call left in it; the MoE kernel
+    // needs its counters at zero when it starts, so clear them on the stream
+    // first (a memset node, no allocation).
+    Q8_CUDA_TRY(cudaMemsetAsync(scratch, 0, moe_ctr_bytes(H), (cudaStream_t)stream));
     return q8_moe_gemv(gate_up_experts, down_experts, shared_gate_up, shared_down, idx, w, x, y, T,
                        E, top_k, H, I, I_shared, scratch, need, stream);
 }
