@@ -52,6 +52,7 @@
 
 #include <stddef.h>
 #include <stdint.h>
+#include <string.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -132,6 +133,35 @@ q8_status q8_unpack_weights(const void *packed, int64_t M, int64_t K, void *gguf
  * below 2^-121 lose relative accuracy there; non-finite x is undefined. */
 q8_status q8_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
                   q8_stream_t stream);
+
+/* Greedy-decode head: the GEMV of q8_gemv with the arg-max over the M outputs
+ * of each column fused into it, so the logits need not be written or read
+ * back ("skuznetsov/cogni-ml" README, its "resident top1" decode step; ties go
+ * to the earliest index, as in the "fusedtok 1.3.0" "API stability" note).
+ * best: [N] uint64 keys, device, 8-byte aligned, overwritten (a first small
+ * kernel on `stream` zeroes them, then the GEMV's CTAs combine theirs with
+ * atomicMax; two launches, both in the dependent-launch chain).  Key =
+ * (order-preserving bits of the max value) << 32 | (0xFFFFFFFF - index): the
+ * row index is q8_argmax_index(key), the value q8_argmax_value(key).  Among
+ * equal values the lowest index wins; -0 counts as +0; NaN outputs are
+ * undefined.  y: [N][M] fp32, or NULL to skip writing the logits; when given
+ * it holds the logits the pick was taken from (best[n] is exactly the first
+ * maximum of y[n]); they meet q8_gemv's tolerance, and match q8_gemv's bits
+ * wherever q8_gemv takes the same column-owner kernel (large M).
+ * 1 <= N <= 4 (larger N -> Q8_ERR_UNSUPPORTED). */
+q8_status q8_gemv_argmax(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                         uint64_t *best, q8_stream_t stream);
+
+static inline int32_t q8_argmax_index(uint64_t key) {
+    return (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFu));
+}
+static inline float q8_argmax_value(uint64_t key) {
+    const uint32_t h = (uint32_t)(key >> 32);
+    const uint32_t u = (h & 0x80000000u) ? (h & 0x7FFFFFFFu) : ~h;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
 
 /* ---------------------------------------------------------------------- */
 /* S4  Fused gate_up + SwiGLU                                              */

@@ -122,6 +122,17 @@ def gemv(gguf, x, M: int, K: int, N: int | None = None, threads: int = 1):
     return y, ya
 
 
+def gemv_argmax(gguf, x, M: int, K: int, threads: int = 1):
+    """O8: greedy pick after the O1 GEMV: for each activation row n, the index
+    of the largest y[n, m], the lowest such index when several are equal (the
+    "resident top1" step of the "skuznetsov/cogni-ml" README; earliest-index
+    ties as in "fusedtok 1.3.0", "API stability").  Returns (idx [N] int64,
+    y, y_abs) with y, y_abs from gemv()."""
+    y, ya = gemv(gguf, x, M, K, threads=threads)
+    # numpy's argmax returns the first occurrence of the maximum
+    return np.argmax(y, axis=1).astype(np.int64), y, ya
+
+
 def gate_up_swiglu(gguf, x, I: int, K: int, threads: int = 1):
     """O2: h = silu(g) * u with g = rows [0, I), u = rows [I, 2I) of W.
 

@@ -19,6 +19,7 @@ import threading
 __all__ = [
     "Q8Error", "lib_path", "q8_status_string", "q8_last_cuda_error", "q8_read_device_error",
     "q8_version", "q8_packed_bytes", "q8_pack_weights", "q8_unpack_weights", "q8_gemv",
+    "q8_gemv_argmax", "q8_argmax_index", "q8_argmax_value",
     "q8_gate_up_swiglu", "q8_moe_route", "q8_moe_workspace_bytes", "q8_moe_workspace_init",
     "q8_moe_gemv",
     "q8_moe_gemv_noalloc",
@@ -44,6 +45,7 @@ _SIGS = {
     "q8_pack_weights": (_INT, [_P, _I64, _I64, _P, _P]),
     "q8_unpack_weights": (_INT, [_P, _I64, _I64, _P, _P]),
     "q8_gemv": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
+    "q8_gemv_argmax": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "q8_gate_up_swiglu": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "q8_moe_route": (_INT, [_P, _I64, _I64, _I64, _INT, _P, _P, _P]),
     "q8_moe_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64, _I64, _I64]),
@@ -148,6 +150,30 @@ def q8_unpack_weights(packed, M, K, gguf_blocks, stream=None):
 
 def q8_gemv(W, x, y, M, K, N, stream=None):
     _call("q8_gemv", _ptr(W), _ptr(x), _ptr(y), M, K, N, _stream(stream))
+
+
+def q8_gemv_argmax(W, x, y, M, K, N, best, stream=None):
+    """y may be None (logits not written); best: [N] uint64 keys (torch.int64
+    or uint64 tensor), decoded by q8_argmax_index / q8_argmax_value."""
+    _call("q8_gemv_argmax", _ptr(W), _ptr(x), None if y is None else _ptr(y), M, K, N, _ptr(best),
+          _stream(stream))
+
+
+def q8_argmax_index(keys):
+    """Row index held in q8_gemv_argmax keys (numpy array or scalar; the
+    header's q8_argmax_index)."""
+    import numpy as np
+    k = np.asarray(keys).astype(np.uint64)
+    return (np.uint64(0xFFFFFFFF) - (k & np.uint64(0xFFFFFFFF))).astype(np.int64)
+
+
+def q8_argmax_value(keys):
+    """Maximum value held in q8_gemv_argmax keys, as float32 (the header's
+    q8_argmax_value)."""
+    import numpy as np
+    h = (np.asarray(keys).astype(np.uint64) >> np.uint64(32)).astype(np.uint32)
+    u = np.where(h & np.uint32(0x80000000), h & np.uint32(0x7FFFFFFF), ~h).astype(np.uint32)
+    return u.view(np.float32)
 
 
 def q8_gate_up_swiglu(W, x, h, I, K, N, stream=None):

@@ -303,10 +303,13 @@ static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_ou
 #endif
 constexpr int64_t kFmMinN = Q8_FM_MIN_N;  // smallest N of fp32 activations sent to the tensor cores
 
+// `best` (fp32 GEMV, N <= 4 only): also leave the arg-max key of every
+// column there (q8_gemv_argmax); the column-owner kernel serves it.
 static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, float *y,
-                          int64_t rows_out, int64_t K, int64_t N, int mode, cudaStream_t stream) {
+                          int64_t rows_out, int64_t K, int64_t N, int mode, cudaStream_t stream,
+                          unsigned long long *best = nullptr) {
     const bool swiglu = mode == kModeSwiGLU;
-    if (mode != kModeQ8Q8 && N >= kFmMinN)
+    if (mode != kModeQ8Q8 && N >= kFmMinN && !best)
         return run_fm(W, static_cast<const float *>(x), y, rows_out, K, N, swiglu, stream);
     const DeviceInfo *dev = nullptr;
     Q8_CHECK(device_info(&dev));
@@ -315,13 +318,14 @@ static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, floa
     const int64_t total_groups = swiglu ? 2 * units : units;
     {
         TilePlan rp;
-        if (plan_resident(units, C, N, mode, dev->sms, &rp) && rp.smem <= (size_t)dev->max_smem_optin &&
+        if (!best && plan_resident(units, C, N, mode, dev->sms, &rp) && rp.smem <= (size_t)dev->max_smem_optin &&
             (uint64_t)units * (uint64_t)rp.grid < (1ull << 31))
             return run_resident(rp, W, static_cast<const float *>(x), y, rows_out, K, N, mode, stream);
     }
     TilePlan p = plan_tile(units, C, N, mode, dev->sms);
     TileArgs &a = p.a;
     a.y = y;
+    a.best = best;
     a.xd = xd;
     a.M_out = (int)rows_out;
     a.up_group0 = swiglu ? (int)units : 0;
@@ -707,6 +711,23 @@ q8_status q8_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K,
     Q8_CHECK(check_device_ptr(x));
     Q8_CHECK(check_device_ptr(y));
     return run_tile(W, x, nullptr, y, M, K, N, kModeF32, (cudaStream_t)stream);
+}
+
+q8_status q8_gemv_argmax(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                         uint64_t *best, q8_stream_t stream) {
+    if (M <= 0 || K <= 0 || N <= 0 || K % 32) return Q8_ERR_SHAPE;
+    if (N > 4 || M > (int64_t)1 << 30 || K > (int64_t)1 << 24) return Q8_ERR_UNSUPPORTED;
+    Q8_CHECK(check_device_ptr(W));
+    Q8_CHECK(check_device_ptr(x));
+    if (y) Q8_CHECK(check_device_ptr(y));
+    Q8_CHECK(check_device_ptr(best, false));
+    if (reinterpret_cast<uintptr_t>(best) & 7u) return Q8_ERR_ALIGN;
+    // the GEMV's CTAs combine their keys with atomicMax, starting from zero
+    Q8_CHECK(launch_pdl(clear_keys_kernel, dim3(1), dim3(32), 0, (cudaStream_t)stream,
+                        "q8_gemv_argmax clear launch", reinterpret_cast<unsigned long long *>(best),
+                        (int)N));
+    return run_tile(W, x, nullptr, y, M, K, N, kModeF32, (cudaStream_t)stream,
+                    reinterpret_cast<unsigned long long *>(best));
 }
 
 q8_status q8_gate_up_swiglu(const void *W, const float *x, float *h, int64_t I, int64_t K,

@@ -41,7 +41,8 @@ constexpr int kTileThreads = (kConsumerWarps + 1) * 32;
 constexpr int kModeF32 = 0, kModeSwiGLU = 1, kModeQ8Q8 = 2;
 
 struct TileArgs {
-    float *y;            // [N][M_out]
+    float *y;            // [N][M_out] (may be null when best is set)
+    unsigned long long *best;  // arg-max keys [N] (q8_gemv_argmax; null otherwise)
     const uint16_t *xd;  // Q8Q8: activation scales [N][B] (read through L1)
     int M_out;           // output rows
     int N;               // activation columns
@@ -168,11 +169,31 @@ template <int NMAX, int MODE>
 __device__ __forceinline__ void store_unit(const TileArgs &a, int unit, int r, const float *v0,
                                            const float *v1) {
     const int row = unit * kGroupRows + r;
-    if (row >= a.M_out) return;
+    if (row >= a.M_out || !a.y) return;
 #pragma unroll
     for (int n = 0; n < NMAX; ++n)
         if (n < a.N)
             a.y[(size_t)n * a.M_out + row] = MODE == kModeSwiGLU ? silu_mul(v0[n], v1[n]) : v0[n];
+}
+
+// Arg-max key of output value v at row `row`: the float's bits mapped to an
+// unsigned order (negative values below positive ones, -0 taken as +0) in
+// the high word, 0xFFFFFFFF - row in the low word, so the largest key is the
+// largest value and, among equal values, the lowest row.
+__device__ __forceinline__ unsigned long long argmax_key(float v, int row) {
+    const uint32_t u = __float_as_uint(v + 0.0f);
+    const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((unsigned long long)ord << 32) | (0xFFFFFFFFu - (uint32_t)row);
+}
+
+// Zeroes the n arg-max keys of q8_gemv_argmax ahead of its GEMV, as a kernel
+// of the dependent-launch chain (a memset node would stop the GEMV from
+// starting early): it waits for the previous grid, which may still combine
+// keys into the same buffer, clears them, and lets the GEMV proceed.
+__global__ void clear_keys_kernel(unsigned long long *keys, int n) {
+    pdl_wait();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = 0ull;
+    pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
@@ -380,6 +401,9 @@ __global__ void __launch_bounds__(ColsCfg<NMAX, MODE, CW_>::THREADS, 1)
     } else if (warp == CW + 1) {
         // ------------------------------ reducer -------------------------------
         pdl_wait_and_trigger();  // the outputs may still be read by the previous grid
+        unsigned long long bestk[NMAX];  // q8_gemv_argmax: this lane's best key per column
+#pragma unroll
+        for (int n = 0; n < NMAX; ++n) bestk[n] = 0ull;
         for (int tl = 0; tl < n_tiles; ++tl) {
             const int p = tl & 1;
             const bool ok = mbar_wait(redfull0 + 8 * p, (tl >> 1) & 1, abort_flag);
@@ -400,10 +424,31 @@ __global__ void __launch_bounds__(ColsCfg<NMAX, MODE, CW_>::THREADS, 1)
                             v[h][n] = sum;
                         }
                     store_unit<NMAX, MODE>(a, ut + g, rr, v[0], v[H - 1]);
+                    const int row = (ut + g) * kGroupRows + rr;
+                    if (MODE == kModeF32 && a.best && row < a.M_out) {
+#pragma unroll
+                        for (int n = 0; n < NMAX; ++n) {
+                            const unsigned long long k = argmax_key(v[0][n], row);
+                            bestk[n] = k > bestk[n] ? k : bestk[n];
+                        }
+                    }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(redfree0 + 8 * p);
+        }
+        if (MODE == kModeF32 && a.best) {
+            // one atomic per column and CTA; the keys were zeroed before the launch
+#pragma unroll
+            for (int n = 0; n < NMAX; ++n) {
+                unsigned long long k = bestk[n];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const unsigned long long t = __shfl_xor_sync(0xffffffffu, k, o);
+                    k = t > k ? t : k;
+                }
+                if (lane == 0 && n < a.N && k != 0ull) atomicMax(a.best + n, k);
+            }
         }
     } else {
         // ------------------------------ consumers -----------------------------

@@ -2,6 +2,7 @@
 
     python -m q8_block_quantized_02_b200.profile --op gemv --M 151936 --K 896 --N 1
     python -m q8_block_quantized_02_b200.profile --op q8q8 --M 37888 --K 3584 --N 16
+    python -m q8_block_quantized_02_b200.profile --op argmax --M 151936 --K 896 --N 1
     python -m q8_block_quantized_02_b200.profile --op moe --T 1
     python -m q8_block_quantized_02_b200.profile --op readpeak
 
@@ -45,9 +46,10 @@ if ROOT not in sys.path:
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--op", choices=["gemv", "swiglu", "q8q8", "moe", "readpeak"], default="gemv",
-                    help="q8_gemv, q8_gate_up_swiglu (M = rows of the stacked gate|up matrix) "
-                         "or q8_quantize_act + q8q8_gemv (only q8q8_gemv is timed)")
+    ap.add_argument("--op", choices=["gemv", "argmax", "swiglu", "q8q8", "moe", "readpeak"], default="gemv",
+                    help="q8_gemv, q8_gemv_argmax (logits not written), q8_gate_up_swiglu (M = rows of "
+                         "the stacked gate|up matrix) or q8_quantize_act + q8q8_gemv (only q8q8_gemv is "
+                         "timed)")
     ap.add_argument("--M", type=int, default=151936)
     ap.add_argument("--K", type=int, default=896)
     ap.add_argument("--N", type=int, default=1)
@@ -94,6 +96,8 @@ def main(argv=None) -> int:
         y = torch.empty((N, M // 2), dtype=torch.float32, device=dev)
     else:
         y = torch.empty((N, M), dtype=torch.float32, device=dev)
+    if args.op == "argmax":
+        best = torch.empty((N,), dtype=torch.int64, device=dev)
     if args.op == "q8q8":
         xq = torch.empty((N, K), dtype=torch.int8, device=dev)
         xd = torch.empty((N, K // 32), dtype=torch.int16, device=dev)
@@ -106,6 +110,8 @@ def main(argv=None) -> int:
         it[0] += 1
         if args.op == "gemv":
             q8.q8_gemv(p, xf, y, M, K, N)
+        elif args.op == "argmax":
+            q8.q8_gemv_argmax(p, xf, None, M, K, N, best)
         elif args.op == "swiglu":
             q8.q8_gate_up_swiglu(p, xf, y, M // 2, K, N)
         else:

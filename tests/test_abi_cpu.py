@@ -14,10 +14,20 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "q8.h")
 
 
+def _header_text() -> str:
+    return re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+
+
+def _inline_helpers() -> list[str]:
+    """static inline functions the header defines (decoders; not exported)."""
+    return sorted(set(re.findall(r"static\s+inline\s+[\w\s\*]*?\b(q8\w*)\s*\(", _header_text())))
+
+
 def _declared_functions() -> list[str]:
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(q8\w*)\s*\(", text)))
+    """Entry points the library must export: every q8* function the header
+    names, less its static inline helpers."""
+    names = set(re.findall(r"\b(q8\w*)\s*\(", _header_text()))
+    return sorted(names - set(_inline_helpers()))
 
 
 @pytest.fixture(scope="module")
@@ -45,8 +55,32 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_binding_covers_the_header():
     import q8_block_quantized_02_b200 as q8
-    for n in _declared_functions():
+    for n in _declared_functions() + _inline_helpers():
         assert hasattr(q8, n), f"python binding lacks {n}"
+
+
+def test_argmax_key_decoders():
+    """The header's key layout: order-preserving float bits high, 0xFFFFFFFF -
+    index low; the binding's decoders invert it for every sign and size."""
+    import numpy as np
+    import q8_block_quantized_02_b200 as q8
+    assert "q8_argmax_index" in _inline_helpers() and "q8_argmax_value" in _inline_helpers()
+    vals = np.array([0.0, 1.5, -1.5, 3.4e38, -3.4e38, 1e-45, -1e-45, 7.0], np.float32)
+    idx = np.array([0, 1, 151935, 7, 2**30, 12, 13, 5], np.int64)
+    u = vals.view(np.uint32).astype(np.uint64)
+    ordered = np.where(u & 0x80000000, ~u & 0xFFFFFFFF, u | 0x80000000)
+    keys = (ordered << np.uint64(32)) | (np.uint64(0xFFFFFFFF) - idx.astype(np.uint64))
+    assert np.array_equal(q8.q8_argmax_index(keys), idx)
+    assert np.array_equal(q8.q8_argmax_value(keys).view(np.uint32), vals.view(np.uint32))
+    # larger value -> larger key (pairwise; +0 and the subnormals included)
+    for i in range(len(vals)):
+        for j in range(len(vals)):
+            if vals[i] > vals[j]:
+                assert int(keys[i]) > int(keys[j])
+    # equal values: the lower index has the larger key
+    k_lo = (np.uint64(0x80000000 | 0x3FC00000) << np.uint64(32)) | np.uint64(0xFFFFFFFF - 3)
+    k_hi = (np.uint64(0x80000000 | 0x3FC00000) << np.uint64(32)) | np.uint64(0xFFFFFFFF - 9)
+    assert k_lo > k_hi and q8.q8_argmax_index(np.array([k_lo]))[0] == 3
 
 
 def test_packed_bytes(lib):

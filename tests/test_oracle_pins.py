@@ -205,6 +205,32 @@ def test_row_and_column_orientation():
     assert np.array_equal(y, [[1, 10], [2, 20], [3, 30]])
 
 
+def test_argmax_closed_forms():
+    """O8 against brute force: with unit scales and one-hot x the outputs are a
+    column of q, so the pick is found by scanning that column for its first
+    maximum by hand; equal rows give the earliest; all-negative columns pick
+    the value nearest zero; several activation rows pick independently."""
+    M, K = 40, 64
+    rng = np.random.default_rng(17)
+    q = rng.integers(-127, 128, (M, K), dtype=np.int8)
+    q[3, 5] = q[21, 5] = q[33, 5] = 127          # three-way tie at the maximum of column 5
+    q[:, 9] = -rng.integers(1, 128, M)           # column 9 all negative
+    q[:, 9][[11, 30]] = -1                       # ... its maximum (-1) twice
+    g = q8gen.assemble_gguf(q, np.full((M, K // 32), 0x3C00, np.uint16))
+    cols = [5, 9, 0, 63]
+    x = np.zeros((len(cols), K), np.float32)
+    for n, k in enumerate(cols):
+        x[n, k] = 1.0
+    idx, y, _ = oracle.gemv_argmax(g, x, M, K)
+    for n, k in enumerate(cols):
+        best = 0
+        for m in range(1, M):
+            if int(q[m, k]) > int(q[best, k]):
+                best = m
+        assert idx[n] == best
+    assert idx[0] == 3 and idx[1] == 11
+
+
 # --------------------------------------------------------------------------
 # P3: linearity in d and x
 # --------------------------------------------------------------------------
