@@ -285,6 +285,24 @@ q8_status q8_moe_gemv_noalloc(const void *gate_up_experts, const void *down_expe
 q8_status q8_quantize_act(const float *x, int8_t *xq, uint16_t *xd, int64_t N, int64_t K,
                           q8_stream_t stream);
 
+/* RMSNorm fused in front of the quantiser (the prologue of the integer
+ * product; the norm that precedes every Qwen projection, "augur" README,
+ * "Features"; "fusedtok 1.3.0" rmsnorm(x, w, eps)).  Per row n:
+ *   r = 1 / sqrt(sum_k x^2 / K + eps), fp32, the sum taken in a fixed order
+ *   inside one CTA (no cross-CTA reduction: the race of "Add Qwen1.5-MoE Q8_0
+ *   ... - #144", conversation), the division, add and reciprocal square root
+ *   correctly rounded;
+ *   xhat[k] = (x[k] * r) * gamma[k], two fp32 roundings in that order;
+ *   xq, xd = the q8_quantize_act rule applied to xhat.
+ * x: [N][K] fp32, 16-byte aligned.  gamma: [K] fp32.  xq: [N][K] int8.
+ * xd: [N][K/32] binary16 bits.  rinv: [N] fp32, the r of each row, or NULL.
+ * Given r, xq and xd are bit-exact; r is within 2^-20 (relative) of the exact
+ * value.  eps must be >= 0 and finite (else Q8_ERR_INVALID); a zero row with
+ * eps == 0, or non-finite x or gamma, gives undefined codes. */
+q8_status q8_rmsnorm_quantize_act(const float *x, const float *gamma, float eps, int8_t *xq,
+                                  uint16_t *xd, float *rinv, int64_t N, int64_t K,
+                                  q8_stream_t stream);
+
 /* ---------------------------------------------------------------------- */
 /* S8  Q8_0 x Q8_0 integer product                                         */
 /* ---------------------------------------------------------------------- */

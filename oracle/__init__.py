@@ -201,6 +201,27 @@ def quantize_act(x, K: int | None = None):
     return q, d, d32
 
 
+def rmsnorm_quantize_act(x, gamma, eps: float, r=None):
+    """O9: RMSNorm then the O5 quantiser.  r_exact[n] = 1 / sqrt(mean_k x^2 +
+    eps) in fp64 (the RMSNorm before every Qwen projection, "augur" README,
+    "Features"; "fusedtok 1.3.0" rmsnorm(x, w, eps)).  The codes are taken
+    from xhat = (x * r) * gamma with two fp32 roundings in that order, where r
+    is the given fp32 per-row factor (the kernel's own; by default r_exact
+    rounded to fp32), so a quantised code is decided in the kernel's
+    precision.  Returns (r_exact fp64 [N], xhat fp32 [N][K], q, d, d32) with
+    q, d, d32 from quantize_act(xhat)."""
+    x = _f32(x).reshape(-1, np.asarray(gamma).size)
+    gamma = _f32(gamma).reshape(-1)
+    x64 = x.astype(np.float64)
+    eps64 = float(np.float32(eps))
+    r_exact = 1.0 / np.sqrt(np.mean(x64 * x64, axis=1) + eps64)
+    r32 = r_exact.astype(np.float32) if r is None else _f32(r).reshape(-1)
+    xhat = (x * r32[:, None]).astype(np.float32)          # fp32 product, round to nearest
+    xhat = (xhat * gamma[None, :]).astype(np.float32)     # then the gain, another rounding
+    q, d, d32 = quantize_act(xhat)
+    return r_exact, xhat, q, d, d32
+
+
 def q8q8(gguf, xq, xd, M: int, K: int, want_dots: bool = True, threads: int = 1):
     """O6: int32 block dots and y = sum_b d_w d_x dot_b (fp64).
 

@@ -23,7 +23,7 @@ __all__ = [
     "q8_gate_up_swiglu", "q8_moe_route", "q8_moe_workspace_bytes", "q8_moe_workspace_init",
     "q8_moe_gemv",
     "q8_moe_gemv_noalloc",
-    "q8_quantize_act", "q8q8_gemv", "q8q8_block_dots",
+    "q8_quantize_act", "q8_rmsnorm_quantize_act", "q8q8_gemv", "q8q8_block_dots",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -56,6 +56,7 @@ _SIGS = {
                                    _I64, _P]),
     "q8_quantize_act": (_INT, [_P, _P, _P, _I64, _I64, _P]),
     "q8q8_gemv": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "q8_rmsnorm_quantize_act": (_INT, [_P, _P, ctypes.c_float, _P, _P, _P, _I64, _I64, _P]),
     "q8q8_block_dots": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
 }
 
@@ -209,6 +210,12 @@ def q8_moe_gemv_noalloc(gate_up_experts, down_experts, shared_gate_up, shared_do
 
 def q8_quantize_act(x, xq, xd, N, K, stream=None):
     _call("q8_quantize_act", _ptr(x), _ptr(xq), _ptr(xd), N, K, _stream(stream))
+
+
+def q8_rmsnorm_quantize_act(x, gamma, eps, xq, xd, rinv, N, K, stream=None):
+    """rinv may be None."""
+    _call("q8_rmsnorm_quantize_act", _ptr(x), _ptr(gamma), float(eps), _ptr(xq), _ptr(xd), _ptr(rinv),
+          N, K, _stream(stream))
 
 
 def q8q8_gemv(W, xq, xd, y, M, K, N, stream=None):

@@ -755,6 +755,26 @@ q8_status q8_quantize_act(const float *x, int8_t *xq, uint16_t *xd, int64_t N, i
                       (cudaStream_t)stream, "q8_quantize_act launch", x, xq, xd, N, K);
 }
 
+q8_status q8_rmsnorm_quantize_act(const float *x, const float *gamma, float eps, int8_t *xq,
+                                  uint16_t *xd, float *rinv, int64_t N, int64_t K, q8_stream_t stream) {
+    if (N <= 0 || K <= 0 || K % 32) return Q8_ERR_SHAPE;
+    if (N > (int64_t)1 << 20 || K > (int64_t)1 << 24) return Q8_ERR_UNSUPPORTED;
+    if (!(eps >= 0.0f) || eps > 3.0e38f) return Q8_ERR_INVALID;  // negative, NaN or infinite
+    Q8_CHECK(check_device_ptr(x));
+    Q8_CHECK(check_device_ptr(gamma, false));
+    Q8_CHECK(check_device_ptr(xq, false));
+    Q8_CHECK(check_device_ptr(xd, false));
+    if ((reinterpret_cast<uintptr_t>(gamma) & 3u) || (reinterpret_cast<uintptr_t>(xd) & 1u))
+        return Q8_ERR_ALIGN;
+    if (rinv) {
+        Q8_CHECK(check_device_ptr(rinv, false));
+        if (reinterpret_cast<uintptr_t>(rinv) & 3u) return Q8_ERR_ALIGN;
+    }
+    return launch_pdl(rmsnorm_quantize_kernel, dim3((unsigned)N), dim3(kRmsThreads), 0,
+                      (cudaStream_t)stream, "q8_rmsnorm_quantize_act launch", x, gamma, eps, xq, xd,
+                      rinv, K);
+}
+
 q8_status q8q8_gemv(const void *W, const int8_t *xq, const uint16_t *xd, float *y, int64_t M,
                     int64_t K, int64_t N, q8_stream_t stream) {
     if (M <= 0 || K <= 0 || N <= 0 || K % 32) return Q8_ERR_SHAPE;

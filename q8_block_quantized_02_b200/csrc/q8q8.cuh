@@ -59,6 +59,67 @@ __global__ void quantize_act_kernel(const float *__restrict__ x, int8_t *__restr
     }
 }
 
+// RMSNorm in front of the quantiser (the norm that precedes every Qwen
+// projection: "augur" README, "Features"), one CTA per activation row so the
+// sum of squares never leaves the CTA (the cross-work-group reduction race of
+// "Add Qwen1.5-MoE Q8_0 ... - #144", conversation): fp32 squares summed
+// per thread with FMA, then across lanes and warps in a fixed order;
+// r = 1 / sqrt(sum / K + eps), correctly rounded; xhat = (x * r) * gamma, two
+// fp32 roundings in that order ("augur" README, "Kernels": fp32 accumulate,
+// the reference's cast order); then each 32-block of xhat is quantised by the
+// rule of quantize_act_kernel, one warp per block (lane i takes element i).
+constexpr int kRmsThreads = 256;
+
+__global__ void __launch_bounds__(kRmsThreads) rmsnorm_quantize_kernel(
+    const float *__restrict__ x, const float *__restrict__ gamma, float eps, int8_t *__restrict__ xq,
+    uint16_t *__restrict__ xd, float *__restrict__ rinv, int64_t K) {
+    __shared__ float part[kRmsThreads / 32];
+    __shared__ float r_s;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t n = blockIdx.x;
+    const float *xr = x + n * K;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    float ss = 0.0f;
+    for (int64_t i = t; i < K / 4; i += kRmsThreads) {
+        const float4 v = reinterpret_cast<const float4 *>(xr)[i];
+        ss = fmaf(v.x, v.x, ss);
+        ss = fmaf(v.y, v.y, ss);
+        ss = fmaf(v.z, v.z, ss);
+        ss = fmaf(v.w, v.w, ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) part[warp] = ss;
+    __syncthreads();
+    if (t == 0) {
+        float sum = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kRmsThreads / 32; ++w) sum += part[w];
+        const float r = __frsqrt_rn(__fadd_rn(__fdiv_rn(sum, (float)K), eps));
+        r_s = r;
+        if (rinv) rinv[n] = r;
+    }
+    __syncthreads();
+    const float r = r_s;
+    const int64_t B = K / 32;
+    for (int64_t b = warp; b < B; b += kRmsThreads / 32) {
+        const float xh = __fmul_rn(__fmul_rn(xr[32 * b + lane], r), gamma[32 * b + lane]);
+        float amax = fabsf(xh);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float d32 = __fdiv_rn(amax, 127.0f);
+        int q = 0;
+        if (d32 != 0.0f) {
+            float rq = roundf(__fdiv_rn(xh, d32));
+            rq = fminf(fmaxf(rq, -127.0f), 127.0f);
+            q = (int)rq;
+        }
+        xq[n * K + 32 * b + lane] = (int8_t)q;
+        if (lane == 0) xd[n * B + b] = __half_as_ushort(__float2half_rn(d32));
+    }
+}
+
 // Test aid: dots[n][m][b] = sum_i q_w[m][32b+i] * xq[n][32b+i], one thread per
 // output, straight from the packed layout.
 __global__ void block_dots_kernel(const uint8_t *__restrict__ W, const int8_t *__restrict__ xq,

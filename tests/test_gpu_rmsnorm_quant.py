@@ -1,0 +1,93 @@
+"""GPU parity of q8_rmsnorm_quantize_act (RMSNorm fused in front of the Q8_0
+activation quantiser, the prologue of the integer product) against the CPU
+oracle, through the C ABI.
+
+The per-row factor r is checked against the exact fp64 value (within 2^-20
+relative); the quantised codes and scales -- integers decided by floating
+point -- are checked bit for bit against the oracle fed the kernel's own r, so
+both sides decide them in the same precision.  The chain RMSNorm -> quantise ->
+Q8 x Q8 product is checked end to end against the oracle's integer product."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+import q8gen
+from q8_test_utils import TOL_REL, assert_within, dev, matrix, pack, torch
+
+pytestmark = pytest.mark.gpu
+
+
+def q8():
+    import q8_block_quantized_02_b200 as m
+    return m
+
+
+def run(x, gamma, eps, with_r=True):
+    t = torch()
+    N, K = x.shape
+    xq = t.empty((N, K), dtype=t.int8, device="cuda")
+    xd = t.empty((N, K // 32), dtype=t.int16, device="cuda")
+    r = t.full((N,), float("nan"), dtype=t.float32, device="cuda") if with_r else None
+    q8().q8_rmsnorm_quantize_act(dev(x), dev(gamma), eps, xq, xd, r, N, K)
+    return (xq.cpu().numpy(), xd.cpu().numpy().view(np.uint16),
+            r.cpu().numpy() if with_r else None)
+
+
+def gain(K, seed):
+    rng = np.random.default_rng(seed)
+    g = (1 + 0.2 * rng.standard_normal(K)).astype(np.float32)
+    g[::97] = 0.0      # a few zero gains
+    g[5::131] *= -1.0  # and some negative ones
+    return g
+
+
+@pytest.mark.parametrize("N,K", [(1, 896), (3, 3584), (16, 4864), (2, 32), (5, 18944), (7, 2048)])
+def test_rmsnorm_quantize_matches_oracle(N, K):
+    x = q8gen.activations(70 + N + K, N, K)
+    x[0, :64] *= 50.0  # an outlier stretch in row 0
+    g = gain(K, K)
+    xq, xd, r = run(x, g, 1e-6)
+    r_exact, _, q_ref, d_ref, _ = oracle.rmsnorm_quantize_act(x, g, 1e-6, r=r)
+    assert np.all(np.abs(r - r_exact) <= 2.0 ** -20 * r_exact)
+    assert np.array_equal(xq, q_ref)
+    assert np.array_equal(xd, d_ref)
+
+
+def test_rmsnorm_quantize_without_r_and_zero_rows():
+    N, K = 4, 1408
+    x = q8gen.activations(71, N, K)
+    x[2] = 0.0  # a zero row: r = 1/sqrt(eps), all codes and scales zero
+    g = gain(K, 3)
+    xq, xd, r = run(x, g, 1e-5)
+    xq2, xd2, _ = run(x, g, 1e-5, with_r=False)
+    assert np.array_equal(xq, xq2) and np.array_equal(xd, xd2)
+    assert np.all(xq[2] == 0) and np.all(xd[2] == 0)
+    assert abs(r[2] - 1e-5 ** -0.5) <= 2.0 ** -20 * 1e-5 ** -0.5
+
+
+def test_rmsnorm_quantize_feeds_the_integer_product():
+    """RMSNorm -> quantise -> q8q8_gemv against the oracle's integer product on
+    the same codes (its tolerance), for a 7B-class gate_up slice."""
+    t = torch()
+    M, K, N = 1024, 3584, 4
+    g_w, _ = matrix(72, M, K)
+    x = q8gen.activations(73, N, K)
+    gam = gain(K, 4)
+    xq, xd, r = run(x, gam, 1e-6)
+    y = t.empty((N, M), dtype=t.float32, device="cuda")
+    q8().q8q8_gemv(pack(g_w, M, K), dev(xq), dev(xd.view(np.int16)), y, M, K, N)
+    _, y_ref, y_abs = oracle.q8q8(g_w, xq, xd, M, K, want_dots=False, threads=oracle.max_threads())
+    assert_within(y.cpu().numpy(), y_ref, TOL_REL * y_abs, "rmsnorm -> q8q8")
+
+
+def test_rmsnorm_quantize_rejects_bad_eps():
+    t = torch()
+    x = np.ones((1, 32), np.float32)
+    xq = t.empty((1, 32), dtype=t.int8, device="cuda")
+    xd = t.empty((1, 1), dtype=t.int16, device="cuda")
+    for eps in (-1e-6, float("nan"), float("inf")):
+        with pytest.raises(q8().Q8Error) as e:
+            q8().q8_rmsnorm_quantize_act(dev(x), dev(np.ones(32, np.float32)), eps, xq, xd, None, 1, 32)
+        assert e.value.status == 1

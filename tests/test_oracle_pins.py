@@ -336,6 +336,37 @@ def test_act_quant_invariants():
 # P7: integer block dots
 # --------------------------------------------------------------------------
 
+def test_rmsnorm_quantize_closed_forms():
+    """O9: a constant row c has r = 1/sqrt(c^2 + eps) (0.5 exactly for c = 2,
+    eps = 0); the row (3, 4, 0, ...) of K = 32 has mean square 25/32, so xhat =
+    (3r, 4r, 0, ...), amax = 4r and the codes are round(95.25) = 95 and 127
+    whatever r rounds to; doubling x halves r and leaves xhat and the codes
+    unchanged (eps = 0); the mean of squares matches exact rationals."""
+    from fractions import Fraction
+    K = 64
+    r, xh, q, d, _ = oracle.rmsnorm_quantize_act(np.full((1, K), 2.0, np.float32), np.ones(K, np.float32), 0.0)
+    assert r[0] == 0.5 and np.all(xh == 1.0) and np.all(q == 127)
+    x = np.zeros((1, 32), np.float32)
+    x[0, 0], x[0, 1] = 3.0, 4.0
+    r, xh, q, d, _ = oracle.rmsnorm_quantize_act(x, np.ones(32, np.float32), 0.0)
+    assert abs(r[0] - (32 / 25) ** 0.5) < 1e-15
+    assert q[0, 0] == 95 and q[0, 1] == 127 and np.all(q[0, 2:] == 0)
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((3, 96)).astype(np.float32)
+    g = (1 + 0.1 * rng.standard_normal(96)).astype(np.float32)
+    r1, xh1, q1, d1, _ = oracle.rmsnorm_quantize_act(x, g, 0.0)
+    r2, xh2, q2, d2, _ = oracle.rmsnorm_quantize_act(2 * x, g, 0.0)
+    assert np.allclose(r2, r1 / 2, rtol=1e-15, atol=0)
+    assert np.array_equal(xh1, xh2) and np.array_equal(q1, q2) and np.array_equal(d1, d2)
+    for n in range(3):
+        ms = sum(Fraction(float(v)) ** 2 for v in x[n]) / 96
+        assert abs(1.0 / r1[n] ** 2 - float(ms)) <= 1e-14 * float(ms)
+    # gamma = 1 and r = 1 reduce O9 to the plain quantiser O5
+    _, _, q3, d3, _ = oracle.rmsnorm_quantize_act(x, np.ones(96, np.float32), 0.0, r=np.ones(3, np.float32))
+    q4, d4, _ = oracle.quantize_act(x)
+    assert np.array_equal(q3, q4) and np.array_equal(d3, d4)
+
+
 def test_int_dots_closed_forms():
     K = 64
     qw = np.full((2, K), 127, np.int8)
