@@ -134,6 +134,18 @@ q8_status q8_unpack_weights(const void *packed, int64_t M, int64_t K, void *gguf
 q8_status q8_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
                   q8_stream_t stream);
 
+/* y[n][m] = (W x)[n][m] + residual[n][m]: the q8_gemv product with the
+ * residual-stream add of the projections that feed it (attention output and
+ * MLP down projection) done in the kernel's store, so the sum costs no extra
+ * pass over y ("fusedtok 1.3.0": fused residual add; the residual adds of the
+ * "skuznetsov/cogni-ml" layer tail).  residual: [N][M] fp32 device; it may be
+ * y itself (in-place update), any other overlap is undefined.  The add is one
+ * fp32 rounding of q8_gemv's own value: bit-identical to adding residual to
+ * the output q8_gemv writes for the same call shape.  Shapes, limits and the
+ * 1e-5 * sum|w x| bound (plus the add's rounding) as q8_gemv. */
+q8_status q8_gemv_residual(const void *W, const float *x, const float *residual, float *y, int64_t M,
+                           int64_t K, int64_t N, q8_stream_t stream);
+
 /* Greedy-decode head: the GEMV of q8_gemv with the arg-max over the M outputs
  * of each column fused into it, so the logits need not be written or read
  * back ("skuznetsov/cogni-ml" README, its "resident top1" decode step; ties go

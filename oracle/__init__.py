@@ -122,6 +122,14 @@ def gemv(gguf, x, M: int, K: int, N: int | None = None, threads: int = 1):
     return y, ya
 
 
+def gemv_residual(gguf, x, residual, M: int, K: int, threads: int = 1):
+    """O10: the O1 GEMV plus a residual stream, y + residual in fp64 (the
+    residual add after the attention output and MLP down projections;
+    "fusedtok 1.3.0" fused residual add).  Returns (y + residual, y_abs)."""
+    y, ya = gemv(gguf, x, M, K, threads=threads)
+    return y + np.asarray(residual, np.float64).reshape(y.shape), ya
+
+
 def gemv_argmax(gguf, x, M: int, K: int, threads: int = 1):
     """O8: greedy pick after the O1 GEMV: for each activation row n, the index
     of the largest y[n, m], the lowest such index when several are equal (the

@@ -124,6 +124,7 @@ struct FmArgs {
     int split;      // CTAs per cluster (K split)
     int stages;
     int up_group0;  // SwiGLU: packed group of the first up row (I / 8)
+    const float *res;  // GEMV: [N][M_out] added to the outputs (q8_gemv_residual; may be y), or null
 };
 
 __device__ __forceinline__ void tmem_ld4_async(uint32_t taddr, uint32_t *v) {
@@ -566,7 +567,10 @@ __global__ void __launch_bounds__(kFmThreads, 1)
                 if (store && active && orow < a.M_out) {
 #pragma unroll
                     for (int t = 0; t < TOK; ++t)
-                        if (n0 + t < a.N) a.y[(size_t)(n0 + t) * a.M_out + orow] = acc[t];
+                        if (n0 + t < a.N) {
+                            const size_t o = (size_t)(n0 + t) * a.M_out + orow;
+                            a.y[o] = a.res ? __fadd_rn(acc[t], a.res[o]) : acc[t];  // y may be res
+                        }
                 }
             }
         }

@@ -275,13 +275,15 @@ static bool plan_resident(int64_t units, int64_t C, int64_t N, int mode, int sms
 }
 
 static q8_status run_resident(const TilePlan &plan, const void *W, const float *x, float *y,
-                              int64_t rows_out, int64_t K, int64_t N, int mode, cudaStream_t stream) {
+                              int64_t rows_out, int64_t K, int64_t N, int mode, cudaStream_t stream,
+                              const float *res) {
     TilePlan p = plan;
     TileArgs &a = p.a;
     const bool swiglu = mode == kModeSwiGLU;
     const int64_t B = K / 32, C = K / 16;
     const int64_t total_groups = swiglu ? 2 * (int64_t)a.units : a.units;
     a.y = y;
+    a.res = res;
     a.M_out = (int)rows_out;
     a.up_group0 = swiglu ? a.units : 0;
     const uint64_t gstride = (uint64_t)kGroupBytesPerBlock * B;
@@ -296,7 +298,7 @@ static q8_status run_resident(const TilePlan &plan, const void *W, const float *
 }
 
 static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_out, int64_t K,
-                        int64_t N, bool swiglu, cudaStream_t stream);
+                        int64_t N, bool swiglu, cudaStream_t stream, const float *res);
 
 #ifndef Q8_FM_MIN_N
 #define Q8_FM_MIN_N 5
@@ -305,12 +307,13 @@ constexpr int64_t kFmMinN = Q8_FM_MIN_N;  // smallest N of fp32 activations sent
 
 // `best` (fp32 GEMV, N <= 4 only): also leave the arg-max key of every
 // column there (q8_gemv_argmax); the column-owner kernel serves it.
+// `res` (fp32 GEMV): added to every output (q8_gemv_residual).
 static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, float *y,
                           int64_t rows_out, int64_t K, int64_t N, int mode, cudaStream_t stream,
-                          unsigned long long *best = nullptr) {
+                          unsigned long long *best = nullptr, const float *res = nullptr) {
     const bool swiglu = mode == kModeSwiGLU;
     if (mode != kModeQ8Q8 && N >= kFmMinN && !best)
-        return run_fm(W, static_cast<const float *>(x), y, rows_out, K, N, swiglu, stream);
+        return run_fm(W, static_cast<const float *>(x), y, rows_out, K, N, swiglu, stream, res);
     const DeviceInfo *dev = nullptr;
     Q8_CHECK(device_info(&dev));
     const int64_t B = K / 32, C = K / 16;
@@ -320,12 +323,13 @@ static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, floa
         TilePlan rp;
         if (!best && plan_resident(units, C, N, mode, dev->sms, &rp) && rp.smem <= (size_t)dev->max_smem_optin &&
             (uint64_t)units * (uint64_t)rp.grid < (1ull << 31))
-            return run_resident(rp, W, static_cast<const float *>(x), y, rows_out, K, N, mode, stream);
+            return run_resident(rp, W, static_cast<const float *>(x), y, rows_out, K, N, mode, stream, res);
     }
     TilePlan p = plan_tile(units, C, N, mode, dev->sms);
     TileArgs &a = p.a;
     a.y = y;
     a.best = best;
+    a.res = res;
     a.xd = xd;
     a.M_out = (int)rows_out;
     a.up_group0 = swiglu ? (int)units : 0;
@@ -492,7 +496,7 @@ static FmPlan plan_fm(int64_t rows_out, int64_t K, int64_t N, bool swiglu, int s
 }
 
 static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_out, int64_t K,
-                        int64_t N, bool swiglu, cudaStream_t stream) {
+                        int64_t N, bool swiglu, cudaStream_t stream, const float *res) {
     const DeviceInfo *dev = nullptr;
     Q8_CHECK(device_info(&dev));
     const int64_t B = K / 32, C = K / 16;
@@ -501,6 +505,7 @@ static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_ou
     FmPlan p = plan_fm(rows_out, K, N, swiglu, dev->sms);
     if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
     p.a.y = y;
+    p.a.res = swiglu ? nullptr : res;
     const uint64_t gstride = (uint64_t)kGroupBytesPerBlock * B;
     const uint8_t *dbase = static_cast<const uint8_t *>(W) + 256 * B;
     CUtensorMap tq, td;
@@ -711,6 +716,19 @@ q8_status q8_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K,
     Q8_CHECK(check_device_ptr(x));
     Q8_CHECK(check_device_ptr(y));
     return run_tile(W, x, nullptr, y, M, K, N, kModeF32, (cudaStream_t)stream);
+}
+
+q8_status q8_gemv_residual(const void *W, const float *x, const float *residual, float *y, int64_t M,
+                           int64_t K, int64_t N, q8_stream_t stream) {
+    if (M <= 0 || K <= 0 || N <= 0 || K % 32) return Q8_ERR_SHAPE;
+    if (N > 16 || M > (int64_t)1 << 30 || K > (int64_t)1 << 24) return Q8_ERR_UNSUPPORTED;
+    Q8_CHECK(check_device_ptr(W));
+    Q8_CHECK(check_device_ptr(x));
+    Q8_CHECK(check_device_ptr(y));
+    Q8_CHECK(check_device_ptr(residual, false));
+    if (reinterpret_cast<uintptr_t>(residual) & 3u) return Q8_ERR_ALIGN;
+    // residual == y is the in-place update; any other overlap is undefined
+    return run_tile(W, x, nullptr, y, M, K, N, kModeF32, (cudaStream_t)stream, nullptr, residual);
 }
 
 q8_status q8_gemv_argmax(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,

@@ -43,6 +43,7 @@ constexpr int kModeF32 = 0, kModeSwiGLU = 1, kModeQ8Q8 = 2;
 struct TileArgs {
     float *y;            // [N][M_out] (may be null when best is set)
     unsigned long long *best;  // arg-max keys [N] (q8_gemv_argmax; null otherwise)
+    const float *res;    // fp32 GEMV: [N][M_out] added to the outputs (q8_gemv_residual; may be y)
     const uint16_t *xd;  // Q8Q8: activation scales [N][B] (read through L1)
     int M_out;           // output rows
     int N;               // activation columns
@@ -172,8 +173,12 @@ __device__ __forceinline__ void store_unit(const TileArgs &a, int unit, int r, c
     if (row >= a.M_out || !a.y) return;
 #pragma unroll
     for (int n = 0; n < NMAX; ++n)
-        if (n < a.N)
-            a.y[(size_t)n * a.M_out + row] = MODE == kModeSwiGLU ? silu_mul(v0[n], v1[n]) : v0[n];
+        if (n < a.N) {
+            const size_t o = (size_t)n * a.M_out + row;
+            a.y[o] = MODE == kModeSwiGLU ? silu_mul(v0[n], v1[n])
+                     : (MODE == kModeF32 && a.res) ? __fadd_rn(v0[n], a.res[o])  // read, then write: y may be res
+                                                   : v0[n];
+        }
 }
 
 // Arg-max key of output value v at row `row`: the float's bits mapped to an
@@ -606,7 +611,7 @@ __device__ __forceinline__ void res_one_group(const uint8_t *smem, const TileArg
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if (lane == 0) {
             const int row = unit * kGroupRows + warp;
-            if (row < a.M_out) a.y[row] = sum;
+            if (row < a.M_out) a.y[row] = a.res ? __fadd_rn(sum, a.res[row]) : sum;
         }
     }
 }

@@ -336,6 +336,21 @@ def test_act_quant_invariants():
 # P7: integer block dots
 # --------------------------------------------------------------------------
 
+def test_gemv_residual_closed_form():
+    """O10: unit scales and one-hot x give a column of q, so y + residual is
+    that column plus the residual, exactly."""
+    M, K = 24, 64
+    rng = np.random.default_rng(9)
+    q = rng.integers(-127, 128, (M, K), dtype=np.int8)
+    g = q8gen.assemble_gguf(q, np.full((M, K // 32), 0x3C00, np.uint16))
+    x = np.zeros((2, K), np.float32)
+    x[0, 7], x[1, 40] = 1.0, 1.0
+    res = rng.standard_normal((2, M)).astype(np.float32)
+    y, _ = oracle.gemv_residual(g, x, res, M, K)
+    assert np.array_equal(y[0], q[:, 7] + res[0].astype(np.float64))
+    assert np.array_equal(y[1], q[:, 40] + res[1].astype(np.float64))
+
+
 def test_rmsnorm_quantize_closed_forms():
     """O9: a constant row c has r = 1/sqrt(c^2 + eps) (0.5 exactly for c = 2,
     eps = 0); the row (3, 4, 0, ...) of K = 32 has mean square 25/32, so xhat =
