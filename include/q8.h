@@ -176,6 +176,32 @@ static inline float q8_argmax_value(uint64_t key) {
 }
 
 /* ---------------------------------------------------------------------- */
+/* K-quant GEMV: Q4_K and Q6_K weights in their raw GGUF layout            */
+/* ---------------------------------------------------------------------- */
+
+/* y[n][m] = sum_k w[m][k] * x[n][k] for a matrix stored as GGUF K-quant
+ * super-blocks of 256 weights (the Q4_K / Q6_K GEMV probes of the
+ * "skuznetsov/cogni-ml" README, "Build Qwen CLIs", which also read the raw
+ * blocks).  W: [M][K/256] blocks, rows contiguous, unpacked.  x: [N][K] fp32,
+ * 16-byte aligned.  y: [N][M] fp32.  K % 256 == 0; 1 <= N <= 4.  Each output
+ * is within 1e-5 * sum_k |w x| of the exact value (every weight formed with
+ * at most one fp32 rounding).  CUDA cores, one warp per row.
+ * Q4_K, 144-byte blocks, W 16-byte aligned: d (binary16) | dmin (binary16) |
+ *   scales[12] | qs[128].  Sub-block j (weights 32j..32j+31) has a 6-bit
+ *   scale sc and min m: j < 4: sc = scales[j] & 63, m = scales[j+4] & 63;
+ *   j >= 4: sc = (scales[j+4] & 15) | (scales[j-4] >> 6) << 4,
+ *   m = (scales[j+4] >> 4) | (scales[j] >> 6) << 4.  Weight e: byte
+ *   qs[32(e/64) + e%32], low nibble if e%64 < 32 else high; w = d sc q - dmin m.
+ * Q6_K, 210-byte blocks: ql[128] | qh[64] | scales[16] (int8) | d (binary16).
+ *   Weight e: h = e/128, c = (e%128)/32, l = e%32; q = ((ql[64h + 32(c&1) + l]
+ *   >> 4(c>>1)) & 15) | ((qh[32h + l] >> 2c) & 3) << 4, minus 32;
+ *   w = d * scales[8h + 2c + l/16] * q. */
+q8_status q8_q4k_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                      q8_stream_t stream);
+q8_status q8_q6k_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                      q8_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
 /* S4  Fused gate_up + SwiGLU                                              */
 /* ---------------------------------------------------------------------- */
 

@@ -74,6 +74,8 @@ def _load():
         lib.oracle_q8q8.restype = None
         lib.oracle_quantize_weights.argtypes = [_P, _I64, _I64, _P, _P]
         lib.oracle_quantize_weights.restype = None
+        lib.oracle_kquant_gemv.argtypes = [ctypes.c_int, _P, _P, _I64, _I64, _I64, _P, _P, _P, ctypes.c_int]
+        lib.oracle_kquant_gemv.restype = None
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -120,6 +122,26 @@ def gemv(gguf, x, M: int, K: int, N: int | None = None, threads: int = 1):
     ya = np.empty((N, M), np.float64)
     _load().oracle_gemv(_ptr(g), _ptr(x), M, K, N, _ptr(y), _ptr(ya), int(threads))
     return y, ya
+
+
+KQ_BYTES = {"q4_k": 144, "q6_k": 210}
+
+
+def kquant_gemv(fmt: str, blocks, x, M: int, K: int, threads: int = 1, want_w: bool = False):
+    """O11: y = W x in fp64 for a raw GGUF Q4_K or Q6_K matrix (the K-quant GEMV
+    probes of the "skuznetsov/cogni-ml" README, "Build Qwen CLIs"); the block
+    packing is written out in q8_oracle.c.  Returns (y, y_abs[, w]) with
+    y_abs = sum_k |w x| and w the dequantised [M][K] weights."""
+    x = _f32(x).reshape(-1, K)
+    N = x.shape[0]
+    b = _u8(blocks)
+    assert K % 256 == 0 and b.size == M * (K // 256) * KQ_BYTES[fmt]
+    y = np.empty((N, M), np.float64)
+    ya = np.empty((N, M), np.float64)
+    w = np.empty((M, K), np.float64) if want_w else None
+    _load().oracle_kquant_gemv(4 if fmt == "q4_k" else 6, _ptr(b), _ptr(x), M, K, N, _ptr(y), _ptr(ya),
+                               _ptr(w), int(threads))
+    return (y, ya, w) if want_w else (y, ya)
 
 
 def gemv_residual(gguf, x, residual, M: int, K: int, threads: int = 1):

@@ -408,3 +408,88 @@ int oracle_max_threads(void) {
     return 1;
 #endif
 }
+
+/* -------------------------------------------------------------------------
+ * K-quant formats (the Q4_K and Q6_K GEMV probes of [cogni-ml], "Build Qwen
+ * CLIs": Q4_K blocks hold "d, dmin, 12-byte packed scales/mins, 128-byte
+ * packed nibbles", Q6_K blocks "ql, qh, signed scales, d").  The pages name
+ * the fields only; the bit packing below is the GGUF one (a reading, listed
+ * in the design doc).  A super-block covers 256 consecutive weights of a row; rows
+ * are contiguous runs of K/256 super-blocks.
+ *
+ * Q4_K, 144 bytes: d (binary16) | dmin (binary16) | scales[12] | qs[128].
+ *   Sub-block j (0..7) covers weights 32j .. 32j+31 and has a 6-bit scale
+ *   sc_j and a 6-bit min m_j:
+ *     j < 4:  sc_j = scales[j] & 63,        m_j = scales[j+4] & 63
+ *     j >= 4: sc_j = (scales[j+4] & 15) | ((scales[j-4] >> 6) << 4)
+ *             m_j  = (scales[j+4] >> 4) | ((scales[j]   >> 6) << 4)
+ *   Weight e (0..255): byte qs[32*(e/64) + e%32], its low nibble when
+ *   (e%64) < 32, else its high nibble; w = d*sc_j*q - dmin*m_j, j = e/32.
+ *
+ * Q6_K, 210 bytes: ql[128] | qh[64] | scales[16] (int8) | d (binary16).
+ *   Weight e: h = e/128, c = (e%128)/32, l = e%32;
+ *     low 4 bits  = ql[64h + 32*(c&1) + l] >> (4*(c>>1)) & 15
+ *     high 2 bits = qh[32h + l] >> (2c) & 3
+ *     q = low | high << 4, minus 32 (so -32..31)
+ *     scale = scales[8h + 2c + l/16];  w = d*scale*q.
+ * ------------------------------------------------------------------------- */
+#define QK_K 256
+#define Q4K_BYTES 144
+#define Q6K_BYTES 210
+
+static double q4k_weight(const uint8_t *blk, int e) {
+    const double d = oracle_half_to_double((uint16_t)(blk[0] | (blk[1] << 8)));
+    const double dmin = oracle_half_to_double((uint16_t)(blk[2] | (blk[3] << 8)));
+    const uint8_t *scales = blk + 4, *qs = blk + 16;
+    const int j = e / 32;
+    int sc, m;
+    if (j < 4) {
+        sc = scales[j] & 63;
+        m = scales[j + 4] & 63;
+    } else {
+        sc = (scales[j + 4] & 15) | ((scales[j - 4] >> 6) << 4);
+        m = (scales[j + 4] >> 4) | ((scales[j] >> 6) << 4);
+    }
+    const uint8_t byte = qs[32 * (e / 64) + e % 32];
+    const int q = (e % 64) < 32 ? (byte & 15) : (byte >> 4);
+    return d * sc * q - dmin * m;
+}
+
+static double q6k_weight(const uint8_t *blk, int e) {
+    const uint8_t *ql = blk, *qh = blk + 128;
+    const int8_t *scales = (const int8_t *)(blk + 192);
+    const double d = oracle_half_to_double((uint16_t)(blk[208] | (blk[209] << 8)));
+    const int h = e / 128, c = (e % 128) / 32, l = e % 32;
+    const int low = (ql[64 * h + 32 * (c & 1) + l] >> (4 * (c >> 1))) & 15;
+    const int high = (qh[32 * h + l] >> (2 * c)) & 3;
+    const int q = (low | (high << 4)) - 32;
+    return d * scales[8 * h + 2 * c + l / 16] * q;
+}
+
+/* y[n][m] = sum_k w[m][k] x[n][k] in fp64 for a K-quant matrix (fmt 4: Q4_K,
+ * 6: Q6_K); y_abs[n][m] = sum_k |w x| (the tolerance scale).  Also the
+ * dequantised weights, when w_out is not NULL ([M][K] fp64). */
+void oracle_kquant_gemv(int fmt, const uint8_t *blocks, const float *x, int64_t M, int64_t K,
+                        int64_t N, double *y, double *y_abs, double *w_out, int nthreads) {
+    const int64_t SB = K / QK_K;
+    const int64_t bytes = fmt == 4 ? Q4K_BYTES : Q6K_BYTES;
+    (void)nthreads;
+#ifdef _OPENMP
+#pragma omp parallel for num_threads(pick_threads(nthreads)) schedule(static)
+#endif
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                const uint8_t *blk = blocks + (m * SB + k / QK_K) * bytes;
+                const double w = fmt == 4 ? q4k_weight(blk, (int)(k % QK_K)) : q6k_weight(blk, (int)(k % QK_K));
+                const double p = w * (double)x[n * K + k];
+                acc += p;
+                aacc += fabs(p);
+                if (w_out && n == 0) w_out[m * K + k] = w;
+            }
+            y[n * M + m] = acc;
+            y_abs[n * M + m] = aacc;
+        }
+    }
+}

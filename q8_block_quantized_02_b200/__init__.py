@@ -20,6 +20,7 @@ __all__ = [
     "Q8Error", "lib_path", "q8_status_string", "q8_last_cuda_error", "q8_read_device_error",
     "q8_version", "q8_packed_bytes", "q8_pack_weights", "q8_unpack_weights", "q8_gemv",
     "q8_gemv_residual", "q8_gemv_argmax", "q8_argmax_index", "q8_argmax_value",
+    "q8_q4k_gemv", "q8_q6k_gemv",
     "q8_gate_up_swiglu", "q8_moe_route", "q8_moe_workspace_bytes", "q8_moe_workspace_init",
     "q8_moe_gemv",
     "q8_moe_gemv_noalloc",
@@ -47,6 +48,8 @@ _SIGS = {
     "q8_gemv": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "q8_gemv_argmax": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "q8_gemv_residual": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "q8_q4k_gemv": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
+    "q8_q6k_gemv": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "q8_gate_up_swiglu": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "q8_moe_route": (_INT, [_P, _I64, _I64, _I64, _INT, _P, _P, _P]),
     "q8_moe_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64, _I64, _I64]),
@@ -152,6 +155,16 @@ def q8_unpack_weights(packed, M, K, gguf_blocks, stream=None):
 
 def q8_gemv(W, x, y, M, K, N, stream=None):
     _call("q8_gemv", _ptr(W), _ptr(x), _ptr(y), M, K, N, _stream(stream))
+
+
+def q8_q4k_gemv(W, x, y, M, K, N, stream=None):
+    """W: raw GGUF Q4_K blocks (uint8 device tensor)."""
+    _call("q8_q4k_gemv", _ptr(W), _ptr(x), _ptr(y), M, K, N, _stream(stream))
+
+
+def q8_q6k_gemv(W, x, y, M, K, N, stream=None):
+    """W: raw GGUF Q6_K blocks (uint8 device tensor)."""
+    _call("q8_q6k_gemv", _ptr(W), _ptr(x), _ptr(y), M, K, N, _stream(stream))
 
 
 def q8_gemv_residual(W, x, residual, y, M, K, N, stream=None):

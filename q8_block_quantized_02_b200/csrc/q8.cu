@@ -13,6 +13,7 @@
 #include "route.cuh"
 #include "tile_gemm.cuh"
 #include "moe.cuh"
+#include "kquant.cuh"
 
 namespace q8 {
 
@@ -638,6 +639,29 @@ static q8_status moe_noalloc_scratch(void **out) {
     return Q8_OK;
 }
 
+template <int FMT>
+// K-quant GEMV launch (kquant.cuh): argument checks, then one warp per row.
+static q8_status run_kquant(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                            cudaStream_t stream, const char *name) {
+    if (M <= 0 || K <= 0 || N <= 0 || K % 256) return Q8_ERR_SHAPE;
+    if (N > 4 || M > (int64_t)1 << 30 || K > (int64_t)1 << 24) return Q8_ERR_UNSUPPORTED;
+    Q8_CHECK(check_device_ptr(W, FMT == 4));  // Q4_K blocks are read as aligned words
+    Q8_CHECK(check_device_ptr(x));
+    Q8_CHECK(check_device_ptr(y, false));
+    if (reinterpret_cast<uintptr_t>(y) & 3u) return Q8_ERR_ALIGN;
+    const DeviceInfo *dev = nullptr;
+    Q8_CHECK(device_info(&dev));
+    const int64_t warps = std::min<int64_t>(M, (int64_t)dev->sms * 64);
+    const unsigned grid = (unsigned)ceil_div(warps, kKqThreads / 32);
+    const int nm = (int)N;
+    const uint8_t *w8 = static_cast<const uint8_t *>(W);
+    switch (nmax_for(N)) {
+        case 1: return launch_pdl(kquant_gemv_kernel<1, FMT>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
+        case 2: return launch_pdl(kquant_gemv_kernel<2, FMT>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
+        default: return launch_pdl(kquant_gemv_kernel<4, FMT>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
+    }
+}
+
 }  // namespace q8
 
 using namespace q8;
@@ -716,6 +740,16 @@ q8_status q8_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K,
     Q8_CHECK(check_device_ptr(x));
     Q8_CHECK(check_device_ptr(y));
     return run_tile(W, x, nullptr, y, M, K, N, kModeF32, (cudaStream_t)stream);
+}
+
+q8_status q8_q4k_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                      q8_stream_t stream) {
+    return run_kquant<4>(W, x, y, M, K, N, (cudaStream_t)stream, "q8_q4k_gemv launch");
+}
+
+q8_status q8_q6k_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                      q8_stream_t stream) {
+    return run_kquant<6>(W, x, y, M, K, N, (cudaStream_t)stream, "q8_q6k_gemv launch");
 }
 
 q8_status q8_gemv_residual(const void *W, const float *x, const float *residual, float *y, int64_t M,

@@ -46,7 +46,8 @@ if ROOT not in sys.path:
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--op", choices=["gemv", "argmax", "swiglu", "q8q8", "moe", "readpeak"], default="gemv",
+    ap.add_argument("--op", choices=["gemv", "argmax", "swiglu", "q8q8", "q4k", "q6k", "moe", "readpeak"],
+                    default="gemv",
                     help="q8_gemv, q8_gemv_argmax (logits not written), q8_gate_up_swiglu (M = rows of "
                          "the stacked gate|up matrix) or q8_quantize_act + q8q8_gemv (only q8q8_gemv is "
                          "timed)")
@@ -78,6 +79,8 @@ def main(argv=None) -> int:
 
     M, K, N = args.M, args.K, args.N
     dev = torch.device("cuda", torch.cuda.current_device())
+    if args.op in ("q4k", "q6k"):
+        return _kquant(args, q8, q8gen, np, torch, dev)
     g, x = q8gen.q8_matrix(args.seed, M, K, N)
     nbytes = q8.q8_packed_bytes(M, K)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -132,6 +135,38 @@ def main(argv=None) -> int:
     weight_bytes = M * K * 34 // 32
     print(json.dumps({"op": args.op, "M": M, "K": K, "N": N, "us_per_call": round(us, 3),
                       "weight_GBps": round(weight_bytes / (us * 1e-6) / 1e9, 1), "copies": copies,
+                      "reps": args.reps, "device_error": word}), flush=True)
+    return 0 if st == 0 else 1
+
+
+def _kquant(args, q8, q8gen, np, torch, dev) -> int:
+    """q8_q4k_gemv / q8_q6k_gemv on raw GGUF K-quant blocks (random fields);
+    bytes per call are the blocks' (144 or 210 per 256 weights)."""
+    M, K, N = args.M, args.K, args.N
+    fmt = "q4_k" if args.op == "q4k" else "q6_k"
+    blocks = q8gen.kquant_matrix(fmt, args.seed, M, K)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = args.copies if args.copies > 0 else max(1, int(np.ceil(3 * l2 / blocks.size)))
+    src = torch.from_numpy(blocks).to(dev)
+    ws = [src.clone() for _ in range(copies)]
+    del src
+    x = torch.from_numpy(q8gen.activations(args.seed + 1, N, K)).to(dev)
+    y = torch.empty((N, M), dtype=torch.float32, device=dev)
+    fn = q8.q8_q4k_gemv if fmt == "q4_k" else q8.q8_q6k_gemv
+    for i in range(args.warmup):
+        fn(ws[i % copies], x, y, M, K, N)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.reps):
+        fn(ws[i % copies], x, y, M, K, N)
+    t1.record()
+    torch.cuda.synchronize()
+    st, word = q8.q8_read_device_error()
+    us = t0.elapsed_time(t1) * 1e3 / max(1, args.reps)
+    print(json.dumps({"op": args.op, "M": M, "K": K, "N": N, "us_per_call": round(us, 3),
+                      "weight_GBps": round(blocks.size / (us * 1e-6) / 1e9, 1), "copies": copies,
                       "reps": args.reps, "device_error": word}), flush=True)
     return 0 if st == 0 else 1
 

@@ -59,6 +59,29 @@ def q8_matrix(seed: int, M: int, K: int, N: int | None = None):
     return gguf, x
 
 
+KQ_BYTES = {"q4_k": 144, "q6_k": 210}
+
+
+def kquant_matrix(fmt: str, seed: int, M: int, K: int) -> np.ndarray:
+    """Raw GGUF K-quant bytes [M][K/256][144 or 210] (flattened uint8): every
+    packed field is uniform random bytes, except the binary16 super-block
+    scales, drawn as |N(0,1)| * 1e-4 (Q4_K d and dmin, bytes 0-3) or
+    |N(0,1)| * 2e-5 (Q6_K d, bytes 208-209), so weights land near the Q8_0
+    recipe's magnitude and some scales are subnormal."""
+    if K % 256:
+        raise ValueError("K must be a multiple of 256")
+    rng = np.random.default_rng(seed)
+    nb = M * (K // 256)
+    b = rng.integers(0, 256, size=(nb, KQ_BYTES[fmt]), dtype=np.uint8)
+    if fmt == "q4_k":
+        dd = (np.abs(rng.standard_normal((nb, 2))) * 1e-4).astype(np.float16)
+        b[:, 0:4] = dd.view(np.uint8).reshape(nb, 4)
+    else:
+        d = (np.abs(rng.standard_normal(nb)) * 2e-5).astype(np.float16)
+        b[:, 208:210] = d.view(np.uint8).reshape(nb, 2)
+    return b.reshape(-1)
+
+
 def activations(seed: int, N: int, K: int) -> np.ndarray:
     """fp32 activations x [N][K] ~ N(0, 1) from their own generator."""
     return np.random.default_rng(seed).standard_normal((N, K)).astype(np.float32)

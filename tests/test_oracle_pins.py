@@ -336,6 +336,89 @@ def test_act_quant_invariants():
 # P7: integer block dots
 # --------------------------------------------------------------------------
 
+# --------------------------------------------------------------------------
+# O11: K-quant formats (Q4_K, Q6_K), against a packer written here from the
+# stated layout (the inverse of the oracle's unpacking) and hand-computed blocks
+# --------------------------------------------------------------------------
+
+def _pack_q4k(d_bits, dmin_bits, sc, m, q):
+    """One Q4_K block from 6-bit scales/mins sc[8], m[8] and nibbles q[256]."""
+    b = np.zeros(144, np.uint8)
+    b[0], b[1] = d_bits & 0xFF, d_bits >> 8
+    b[2], b[3] = dmin_bits & 0xFF, dmin_bits >> 8
+    for j in range(4):
+        b[4 + j] = (sc[j] & 63) | ((sc[j + 4] >> 4) << 6)
+        b[8 + j] = (m[j] & 63) | ((m[j + 4] >> 4) << 6)
+        b[12 + j] = (sc[j + 4] & 15) | ((m[j + 4] & 15) << 4)
+    for e in range(256):
+        i = 16 + 32 * (e // 64) + e % 32
+        b[i] |= (q[e] & 15) << (0 if e % 64 < 32 else 4)
+    return b
+
+
+def _pack_q6k(d_bits, scales, q):
+    """One Q6_K block from int8 scales[16] and q[256] in [-32, 31]."""
+    b = np.zeros(210, np.uint8)
+    for e in range(256):
+        u = int(q[e]) + 32
+        h, c, l = e // 128, (e % 128) // 32, e % 32
+        b[64 * h + 32 * (c & 1) + l] |= (u & 15) << (4 * (c >> 1))
+        b[128 + 32 * h + l] |= (u >> 4) << (2 * c)
+    b[192:208] = np.asarray(scales, np.int8).view(np.uint8)
+    b[208], b[209] = d_bits & 0xFF, d_bits >> 8
+    return b
+
+
+def test_kquant_round_trip():
+    """Random fields packed here decode, in the oracle, to exactly d*sc*q - dmin*m
+    (Q4_K) and d*scale*q (Q6_K) at every position; the GEMV equals the fp64
+    product of those weights."""
+    rng = np.random.default_rng(31)
+    for trial in range(6):
+        dbits, mbits = [int(v) for v in (np.abs(rng.standard_normal(2)) * 0.01).astype(np.float16).view(np.uint16)]
+        sc, m = rng.integers(0, 64, 8), rng.integers(0, 64, 8)
+        q = rng.integers(0, 16, 256)
+        blk4 = _pack_q4k(dbits, mbits, sc, m, q)
+        d, dmin = oracle.half_to_double(dbits), oracle.half_to_double(mbits)
+        want4 = np.array([d * sc[e // 32] * q[e] - dmin * m[e // 32] for e in range(256)])
+        x = rng.standard_normal((2, 256)).astype(np.float32)
+        y, _, w = oracle.kquant_gemv("q4_k", blk4, x, 1, 256, want_w=True)
+        assert np.array_equal(w[0], want4)
+        assert np.allclose(y[:, 0], x.astype(np.float64) @ want4, rtol=1e-12, atol=0)
+        scales6 = rng.integers(-128, 128, 16)
+        q6 = rng.integers(-32, 32, 256)
+        blk6 = _pack_q6k(dbits, scales6, q6)
+        want6 = np.array([d * scales6[e // 16] * q6[e] for e in range(256)])
+        y6, _, w6 = oracle.kquant_gemv("q6_k", blk6, x, 1, 256, want_w=True)
+        assert np.array_equal(w6[0], want6)
+        assert np.allclose(y6[:, 0], x.astype(np.float64) @ want6, rtol=1e-12, atol=0)
+
+
+def test_kquant_hand_blocks():
+    """Q4_K: d = 1, dmin = 0.5; scales bytes give sc0 = 3, m0 = 1, sc4 = 53,
+    m4 = 34 (high bits from bytes 0 and 4), all other scales and mins 0; every
+    qs byte 0x21.  Sub-block 0 weights 1*3*1 - 0.5*1 = 2.5, sub-block 4 weights
+    53*1 - 0.5*34 = 36, the rest 0: with x = 1, y = 32*2.5 + 32*36 = 1232.
+    Q6_K: d = 0.25, scales[0] = -3, the others 2; ql bytes 0xFF, qh 0 (q = 15 -
+    32 = -17): weights 12.75 (first 16) and -8.5: y = 204 - 2040 = -1836."""
+    b = np.zeros(144, np.uint8)
+    b[0:4] = [0x00, 0x3C, 0x00, 0x38]
+    b[4] = 0b11000011   # sc0 = 3, top bits of sc4 = 3
+    b[8] = 0b10000001   # m0 = 1, top bits of m4 = 2
+    b[12] = 0x25        # sc4 low = 5, m4 low = 2
+    b[16:] = 0x21
+    y, _, w = oracle.kquant_gemv("q4_k", b, np.ones((1, 256), np.float32), 1, 256, want_w=True)
+    assert y[0, 0] == 1232.0
+    assert np.all(w[0, :32] == 2.5) and np.all(w[0, 128:160] == 36.0)
+    assert np.all(w[0, 32:128] == 0) and np.all(w[0, 160:] == 0)
+    b6 = np.zeros(210, np.uint8)
+    b6[:128] = 0xFF
+    b6[192:208] = np.array([-3] + [2] * 15, np.int8).view(np.uint8)
+    b6[208:210] = [0x00, 0x34]
+    y6, _ = oracle.kquant_gemv("q6_k", b6, np.ones((1, 256), np.float32), 1, 256)
+    assert y6[0, 0] == -1836.0
+
+
 def test_gemv_residual_closed_form():
     """O10: unit scales and one-hot x give a column of q, so y + residual is
     that column plus the residual, exactly."""
