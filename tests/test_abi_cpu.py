@@ -59,6 +59,35 @@ def test_binding_covers_the_header():
         assert hasattr(q8, n), f"python binding lacks {n}"
 
 
+def test_header_compiles_as_c_and_cpp(tmp_path):
+    """include/q8.h is a C ABI: a translation unit using it compiles as strict
+    C99 and as C++, and a C program built on its inline key decoders gives
+    back what a key was made from."""
+    import subprocess
+    if shutil.which("gcc") is None or shutil.which("g++") is None:
+        pytest.skip("gcc / g++ not available")
+    inc = os.path.join(ROOT, "include")
+    uses = tmp_path / "uses_entry_points.c"
+    uses.write_text(
+        '#include "q8.h"\n'
+        "q8_status call_gemv(const void *w, const float *x, float *y) {\n"
+        "  return q8_gemv(w, x, y, 8, 32, 1, (q8_stream_t)0);\n}\n")
+    for cmd in (["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-c"],
+                ["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-x", "c++", "-c"]):
+        subprocess.run(cmd + ["-I", inc, str(uses), "-o", str(tmp_path / "uses.o")], check=True)
+    prog = tmp_path / "decode_key.c"
+    prog.write_text(
+        '#include "q8.h"\n#include <stdio.h>\n'
+        "int main(void) {\n"
+        "  uint64_t k = ((uint64_t)(0x80000000u | 0x3FC00000u) << 32) | (0xFFFFFFFFu - 7u);\n"
+        '  printf("%d %g\\n", q8_argmax_index(k), (double)q8_argmax_value(k));\n'
+        "  return 0;\n}\n")
+    exe = tmp_path / "decode_key"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", inc, str(prog), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out == ["7", "1.5"]
+
+
 def test_argmax_key_decoders():
     """The header's key layout: order-preserving float bits high, 0xFFFFFFFF -
     index low; the binding's decoders invert it for every sign and size."""
