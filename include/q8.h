@@ -148,7 +148,7 @@ q8_status q8_gemv_residual(const void *W, const float *x, const float *residual,
 
 /* Greedy-decode head: the GEMV of q8_gemv with the arg-max over the M outputs
  * of each column fused into it, so the logits need not be written or read
- * back ("skuznetsov/cogni-ml" README, its "resident top1" decode step; ties go
+ * back ("skuznetsov/cogni-ml" README, its resident top-1 decode step; ties go
  * to the earliest index, as in the "fusedtok 1.3.0" "API stability" note).
  * best: [N] uint64 keys, device, 8-byte aligned, overwritten (a first small
  * kernel on `stream` zeroes them, then the GEMV's CTAs combine theirs with

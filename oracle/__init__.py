@@ -155,7 +155,7 @@ def gemv_residual(gguf, x, residual, M: int, K: int, threads: int = 1):
 def gemv_argmax(gguf, x, M: int, K: int, threads: int = 1):
     """O8: greedy pick after the O1 GEMV: for each activation row n, the index
     of the largest y[n, m], the lowest such index when several are equal (the
-    "resident top1" step of the "skuznetsov/cogni-ml" README; earliest-index
+    resident top-1 step of the "skuznetsov/cogni-ml" README; earliest-index
     ties as in "fusedtok 1.3.0", "API stability").  Returns (idx [N] int64,
     y, y_abs) with y, y_abs from gemv()."""
     y, ya = gemv(gguf, x, M, K, threads=threads)

@@ -26,7 +26,7 @@
  *   [fusedtok]  "fusedtok 1.3.0" PKG-INFO, "API stability": selection ties
  *               resolve to the earliest index.
  *
- * Readings where the pages are silent (each also listed in the design doc):
+ * Readings where the pages are silent:
  *   - A Q8_0 block is 34 bytes: a little-endian binary16 scale d, then 32 int8
  *     values q; a weight is d*q.  Blocks run along K, rows are contiguous.
  *   - A fused gate_up matrix has the gate rows first ([0, I)) and the up rows
@@ -411,11 +411,12 @@ int oracle_max_threads(void) {
 
 /* -------------------------------------------------------------------------
  * K-quant formats (the Q4_K and Q6_K GEMV probes of [cogni-ml], "Build Qwen
- * CLIs": Q4_K blocks hold "d, dmin, 12-byte packed scales/mins, 128-byte
- * packed nibbles", Q6_K blocks "ql, qh, signed scales, d").  The pages name
- * the fields only; the bit packing below is the GGUF one (a reading, listed
- * in the design doc).  A super-block covers 256 consecutive weights of a row; rows
- * are contiguous runs of K/256 super-blocks.
+ * CLIs", which lists the fields of each block: for Q4_K two binary16 scales,
+ * twelve bytes of packed 6-bit scales and mins, and 128 bytes of 4-bit
+ * values; for Q6_K low-bit and high-bit value arrays, signed 8-bit scales and
+ * one binary16 scale).  The pages give no bit packing; the one below is the
+ * GGUF one (a reading).  A super-block covers 256 consecutive weights of a
+ * row; rows are contiguous runs of K/256 super-blocks.
  *
  * Q4_K, 144 bytes: d (binary16) | dmin (binary16) | scales[12] | qs[128].
  *   Sub-block j (0..7) covers weights 32j .. 32j+31 and has a 6-bit scale

@@ -20,12 +20,12 @@
 // at once, and the epilogue adds
 //     d_w * s * (D_0 + D_1 / 254 + D_2 / 254^2)
 // into fp32 accumulators.  Each Q8_0 block needs its own weight scale d_w, so
-// one MMA per block, as in the integer path.  (The Q8_0 definition, w = d * q
-// per 32-block, is that of "ggml quantization formats", section Q8_0; the
-// per-block int8 dot followed by the scales is the activation-quantised dot of
-// "Add Qwen1.5-MoE Q8_0 ... - #144", "Key implementation notes", here with an
-// exact three-term split of x in place of the one-term Q8_0 rounding, so the
-// result keeps fp32 accuracy.)
+// one MMA per block, as in the integer path.  (The weights are the raw GGUF
+// Q8_0 blocks of the "skuznetsov/cogni-ml" README's Q8_0 GEMV probe, "Build
+// Qwen CLIs", w = d * q per 32-block; the per-block int8 dot followed by the
+// scales is the activation-quantised dot of "Add Qwen1.5-MoE Q8_0 ... - #144",
+// "Key implementation notes", here with an exact three-term split of x in
+// place of the one-term Q8_0 rounding, so the result keeps fp32 accuracy.)
 //
 // Activation blocks whose largest magnitude is below 2^-121 are scaled as if
 // it were 2^-121 and lose relative accuracy (fp32 subnormal territory).

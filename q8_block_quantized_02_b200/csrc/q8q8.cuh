@@ -65,9 +65,10 @@ __global__ void quantize_act_kernel(const float *__restrict__ x, int8_t *__restr
 // "Add Qwen1.5-MoE Q8_0 ... - #144", conversation): fp32 squares summed
 // per thread with FMA, then across lanes and warps in a fixed order;
 // r = 1 / sqrt(sum / K + eps), correctly rounded; xhat = (x * r) * gamma, two
-// fp32 roundings in that order ("augur" README, "Kernels": fp32 accumulate,
-// the reference's cast order); then each 32-block of xhat is quantised by the
-// rule of quantize_act_kernel, one warp per block (lane i takes element i).
+// fp32 roundings in that order (the "augur" README's Triton RMSNorm, section
+// "Kernels", sums in fp32 and keeps its reference's order of conversions);
+// then each 32-block of xhat is quantised by the rule of quantize_act_kernel,
+// one warp per block (lane i takes element i).
 constexpr int kRmsThreads = 256;
 
 __global__ void __launch_bounds__(kRmsThreads) rmsnorm_quantize_kernel(

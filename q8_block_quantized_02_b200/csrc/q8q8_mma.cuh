@@ -5,9 +5,11 @@
 // A Q8_0 block dot needs its own pair of scales, so the tensor cores take one
 // 32-deep block at a time: D[m][n] = sum_i A[m][i] * xq[n][i] over one block,
 // exact in int32, and the epilogue adds float(dot) * d_w[m] * d_x[n] into fp32
-// registers.  (The Q8_0 definition and the block-dot-then-scale order of the
-// integer path are in "ggml quantization formats", section Q8_0, and in the
-// llama.cpp "vec_dot_q8_0_q8_0" description.)
+// registers.  (The block-dot-then-scale order is the integer path of "Add
+// Qwen1.5-MoE Q8_0 ... - #144", "Key implementation notes": each activation
+// block quantised to int8, then int8 x int8 accumulation with the Q8_0
+// scales; the weights are the raw GGUF Q8_0 blocks of the
+// "skuznetsov/cogni-ml" README's Q8_0 GEMV probe, "Build Qwen CLIs".)
 //
 // Operands straight from the packed layout (include/q8.h):
 //   * A = weights, M = 128 rows (16 packed groups) x K = 32 bytes.  A group's
