@@ -136,3 +136,69 @@ def test_status_strings(lib):
 def test_library_targets_sm100a_only():
     from q8_block_quantized_02_b200 import build
     assert "arch=compute_100a,code=sm_100a" in " ".join(build.NVCC_FLAGS)
+
+
+def test_host_validation_runs_before_any_device_work(lib):
+    """Every entry point checks shapes, size limits, null pointers and flags on
+    the host before it touches CUDA, so these rejections need no GPU: 2 =
+    Q8_ERR_SHAPE, 5 = Q8_ERR_UNSUPPORTED, 1 = Q8_ERR_INVALID."""
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    F = ctypes.c_float
+
+    def fn(name, *argtypes):
+        f = getattr(lib, name)
+        f.restype = ctypes.c_int
+        f.argtypes = list(argtypes)
+        return f
+
+    n = None  # null pointer / default stream
+    gemv = fn("q8_gemv", P, P, P, I64, I64, I64, P)
+    assert gemv(n, n, n, 8, 48, 1, n) == 2          # K % 32
+    assert gemv(n, n, n, 0, 32, 1, n) == 2          # M <= 0
+    assert gemv(n, n, n, 8, 32, 0, n) == 2          # N <= 0
+    assert gemv(n, n, n, 8, 32, 17, n) == 5         # N > 16
+    assert gemv(n, n, n, 8, 32, 1, n) == 1          # null W
+    res = fn("q8_gemv_residual", P, P, P, P, I64, I64, I64, P)
+    assert res(n, n, n, n, 8, 40, 1, n) == 2
+    assert res(n, n, n, n, 8, 32, 17, n) == 5
+    assert res(n, n, n, n, 8, 32, 2, n) == 1
+    am = fn("q8_gemv_argmax", P, P, P, I64, I64, I64, P, P)
+    assert am(n, n, n, 8, 33, 1, n, n) == 2
+    assert am(n, n, n, 8, 32, 5, n, n) == 5         # N > 4
+    assert am(n, n, n, 8, 32, 4, n, n) == 1
+    sw = fn("q8_gate_up_swiglu", P, P, P, I64, I64, I64, P)
+    assert sw(n, n, n, 12, 32, 1, n) == 2           # I % 8
+    assert sw(n, n, n, 16, 32, 17, n) == 5
+    qa = fn("q8_quantize_act", P, P, P, I64, I64, P)
+    assert qa(n, n, n, 1, 31, n) == 2
+    rq = fn("q8_rmsnorm_quantize_act", P, P, F, P, P, P, I64, I64, P)
+    assert rq(n, n, 1e-6, n, n, n, 1, 48, n) == 2
+    assert rq(n, n, -1e-6, n, n, n, 1, 32, n) == 1  # eps < 0
+    assert rq(n, n, float("nan"), n, n, n, 1, 32, n) == 1
+    assert rq(n, n, float("inf"), n, n, n, 1, 32, n) == 1
+    qq = fn("q8q8_gemv", P, P, P, P, I64, I64, I64, P)
+    assert qq(n, n, n, n, 8, 16, 1, n) == 2
+    assert qq(n, n, n, n, 8, 32, 17, n) == 5
+    bd = fn("q8q8_block_dots", P, P, P, I64, I64, I64, P)
+    assert bd(n, n, n, 8, 20, 1, n) == 2
+    for name in ("q8_q4k_gemv", "q8_q6k_gemv"):
+        kq = fn(name, P, P, P, I64, I64, I64, P)
+        assert kq(n, n, n, 8, 896, 1, n) == 2       # K % 256
+        assert kq(n, n, n, 8, 512, 5, n) == 5       # N > 4
+        assert kq(n, n, n, 8, 512, 1, n) == 1
+    route = fn("q8_moe_route", P, I64, I64, I64, ctypes.c_int, P, P, P)
+    assert route(n, 1, 4, 5, 0, n, n, n) == 2       # top_k > E
+    assert route(n, 17, 60, 4, 0, n, n, n) == 5     # T > 16
+    assert route(n, 1, 60, 4, 2, n, n, n) == 1      # renormalize not 0/1
+    moe = fn("q8_moe_gemv", P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, P, ctypes.c_size_t, P)
+    assert moe(n, n, n, n, n, n, n, n, 1, 60, 4, 2000, 1408, 5632, n, 0, n) == 2    # H % 32
+    assert moe(n, n, n, n, n, n, n, n, 1, 60, 4, 2048, 1408, 5632, n, 0, n) == 1    # half a shared expert
+    noalloc = fn("q8_moe_gemv_noalloc", P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, P)
+    assert noalloc(n, n, n, n, n, n, n, n, 16, 64, 8, 2048, 8192, 32, n) == 5      # scratch too small
+    msg = lib.q8_last_cuda_error
+    msg.restype = ctypes.c_char_p
+    assert b"4194304" in msg()
+    pack = fn("q8_pack_weights", P, I64, I64, P, P)
+    assert pack(n, 8, 40, n, n) == 2
+    init = fn("q8_moe_workspace_init", P, ctypes.c_size_t, P)
+    assert init(n, 0, n) == 2
