@@ -129,8 +129,12 @@ q8_status q8_unpack_weights(const void *packed, int64_t M, int64_t K, void *gguf
  * int8 q against an exact three-term int8 split of each 32-block of x,
  * x = s (q0 + q1/254 + q2/254^2) with a power-of-two s per block (residual
  * below 2.5e-7 of the block's max |x|), and an fp32 epilogue applies d and s
- * per block; the same 1e-5 bound holds.  Activation blocks whose max |x| is
- * below 2^-121 lose relative accuracy there; non-finite x is undefined. */
+ * per block.  There the split adds at most 2.5e-7 * sum_b amax_b * sum_{k in b}
+ * |w_k| (amax_b: block b's max |x|) to the fp32 error: within the 1e-5 bar
+ * for ordinary activations (all tests, including blocks of tiny values with
+ * one large one), but not for every crafted input -- e.g. a block whose only
+ * large value meets a zero weight.  Blocks whose max |x| is below 2^-121 lose
+ * relative accuracy there; non-finite x is undefined. */
 q8_status q8_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
                   q8_stream_t stream);
 
