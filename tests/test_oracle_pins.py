@@ -576,3 +576,55 @@ def test_moe_reduces_to_dense():
     dn2 = np.concatenate([dn, dn])
     y3, _, _ = oracle.moe(gu2, dn2, None, None, idx2 + np.array([[0, 1]]), w2, x, H, I, 0)
     assert np.allclose(y3, y * w2.sum(axis=1)[:, None], rtol=1e-12, atol=1e-12 * np.abs(y).max())
+
+
+def _dense_mlp(gu_bytes, dn_bytes, x_row, H, I):
+    """One expert's SwiGLU MLP on one token: h from O2 on that expert's own
+    gate_up bytes, then its down matrix decoded from its GGUF bytes by numpy
+    and applied in fp64."""
+    h = oracle.gate_up_swiglu(gu_bytes, x_row[None, :], I, H)["h"][0]
+    q, dbits = q8gen.split_gguf(dn_bytes, H, I)
+    wd = q.astype(np.float64) * np.repeat(dbits.view(np.float16).astype(np.float64), 32, axis=1)
+    return wd @ h
+
+
+def test_moe_distinct_experts_match_dense_mlps():
+    """O4 with several *different* experts: every token's output is the
+    weighted sum of the dense MLPs of exactly the experts its idx row names,
+    in any slot position, plus the shared expert with weight one (the router +
+    top-k expert + shared-expert FFN block of the GPULlama3.java Qwen1.5-MoE
+    pull request, PR summary).  Each expert's MLP is computed from its own byte
+    slice of the stacked buffers, so reading the wrong expert (a fixed index,
+    the slot number in place of idx, a wrong stride) changes the result."""
+    H, I, Is, E = 64, 96, 64, 5
+    gu_list, dn_list = [], []
+    for e in range(E):
+        gu_list.append(q8gen.q8_matrix(300 + e, 2 * I, H)[0])
+        dn_list.append(q8gen.q8_matrix(400 + e, H, I)[0])
+    sgu = q8gen.q8_matrix(500, 2 * Is, H)[0]
+    sdn = q8gen.q8_matrix(501, H, Is)[0]
+    gu_all, dn_all = np.concatenate(gu_list), np.concatenate(dn_list)
+    x = q8gen.activations(502, 4, H)
+    # distinct experts in different slot positions, one token reusing another's
+    # expert in the other slot, unequal weights
+    idx = np.array([[3, 1, 4], [0, 2, 3], [4, 3, 1], [2, 0, 4]], np.int32)
+    w = np.array([[0.5, 0.25, 0.125], [0.375, 0.0625, 0.3125], [0.2, 0.7, 0.1], [0.9, 0.05, 0.05]])
+    y, bound, slot = oracle.moe(gu_all, dn_all, None, None, idx, w, x, H, I, 0)
+    ys, _, _ = oracle.moe(gu_all, dn_all, sgu, sdn, idx, w, x, H, I, Is)
+    for t in range(idx.shape[0]):
+        want = np.zeros(H)
+        for s in range(idx.shape[1]):
+            e = int(idx[t, s])
+            o = _dense_mlp(gu_list[e], dn_list[e], x[t], H, I)
+            assert np.allclose(slot[t, s], o, rtol=1e-12, atol=1e-12 * np.abs(o).max())
+            want += w[t, s] * o
+        assert np.allclose(y[t], want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+        sh = _dense_mlp(sgu, sdn, x[t], H, Is)
+        assert np.allclose(ys[t], want + sh, rtol=1e-12, atol=1e-12 * np.abs(want + sh).max())
+    # the experts really differ: swapping two picks of a token changes its output
+    idx2 = idx.copy()
+    idx2[0, [0, 1]] = idx2[0, [1, 0]]
+    y2, _, _ = oracle.moe(gu_all, dn_all, None, None, idx2, w, x, H, I, 0)
+    assert np.abs(y2[0] - y[0]).max() > 1e-3 * np.abs(y[0]).max()
+    assert np.array_equal(y2[1:], y[1:])
+    assert np.all(bound > 0)
