@@ -153,6 +153,21 @@ def test_gemv_full_size_sampled(M, K):
     assert_within(y[:, rows], y_ref, TOL_REL * y_abs, f"full-size {M}x{K}")
 
 
+@pytest.mark.parametrize("M,K", [(152064, 3584), (3584, 18944)])
+@pytest.mark.parametrize("N", [2, 4])
+def test_gemv_full_size_sampled_small_batch(M, K, N):
+    """The 7B-class lm_head and down at N = 2 and 4 (the small-batch sweep's
+    CUDA-core columns), full size, at the launch shape the planner picks for
+    them; sampled rows against the oracle."""
+    g, x = matrix(3030 + M + N, M, K, N)
+    y = gemv(pack(g, M, K), x, M, K)
+    rng = np.random.default_rng(N)
+    rows = np.unique(np.concatenate([np.arange(16), np.arange(M - 16, M), rng.integers(0, M, 300),
+                                     np.arange(127, M, 4096)]))
+    y_ref, y_abs = oracle.gemv(rows_subset(g, M, K, rows), x, len(rows), K, threads=oracle.max_threads())
+    assert_within(y[:, rows], y_ref, TOL_REL * y_abs, f"full-size {M}x{K} N={N}")
+
+
 # --------------------------------------------------------------------------
 # S4 fused gate_up + SwiGLU
 # --------------------------------------------------------------------------
@@ -171,12 +186,13 @@ def test_gate_up_swiglu_matches_oracle(I, K, N):
     assert_within(h, ref["h"], swiglu_bound(ref), f"swiglu I={I} K={K} N={N}")
 
 
-def test_gate_up_full_size_sampled():
-    """7B-class gate_up (37888 x 3584) at N = 1, sampled rows."""
+@pytest.mark.parametrize("N", [1, 2, 4])
+def test_gate_up_full_size_sampled(N):
+    """7B-class gate_up (37888 x 3584) at N = 1, 2 and 4, sampled rows."""
     I, K = 18944, 3584
-    g, x = matrix(4242, 2 * I, K, 1)
+    g, x = matrix(4242 + (N - 1) * 7, 2 * I, K, N)
     h = gate_up(pack(g, 2 * I, K), x, I, K)
-    rng = np.random.default_rng(2)
+    rng = np.random.default_rng(2 + N)
     rows = np.unique(np.concatenate([np.arange(8), np.arange(I - 8, I), rng.integers(0, I, 300)]))
     sub = np.concatenate([rows_subset(g, 2 * I, K, rows), rows_subset(g, 2 * I, K, rows + I)])
     ref = oracle.gate_up_swiglu(sub, x, len(rows), K, threads=oracle.max_threads())

@@ -153,6 +153,35 @@ def test_q8q8_tensor_core_deterministic_and_exact_on_integers():
     assert np.array_equal(y.astype(np.float64), y_ref)
 
 
+@pytest.mark.parametrize("M,K,N", [
+    (4096, 896, 1),      # 8-consumer-warp column kernel
+    (4096, 18944, 1),    # 16-warp kernel (a CTA's share of the weights >= 256 KB)
+    (37888, 3584, 1),    # 16-warp kernel, 32 row groups per CTA, two consumer groups
+    (4096, 896, 2),
+    (4096, 18944, 2),
+    (1000, 3584, 3),     # N = 3 on the 4-column build, ragged last group
+    (4096, 18944, 4),
+    (37888, 3584, 4),
+])
+def test_q8q8_cuda_cores_exact_on_integers(M, K, N):
+    """The dp4a kernels (N <= 4): with unit scales every output is the exact
+    integer sum of the int32 block dots (int8 x int8 accumulated exactly, the
+    scales applied per block -- the GPULlama3.java Qwen1.5-MoE pull request,
+    "Key implementation notes"), which fp32 holds exactly while partial sums
+    stay below 2^24; so y must equal the oracle's sum of block dots bit for
+    bit, at the shapes that take the 8- and 16-warp column kernels."""
+    g, x = q8gen.q8_matrix(M + 3 * K + N, M, K, N)
+    xq, _, _ = oracle.quantize_act(x)
+    qw, _ = q8gen.split_gguf(g, M, K)
+    g1 = q8gen.assemble_gguf(qw, np.full((M, K // 32), 0x3C00, np.uint16))
+    xd1 = np.full((N, K // 32), 0x3C00, np.uint16)
+    y = run_q8q8(g1, xq, xd1, M, K)
+    dots, y_ref, _ = oracle.q8q8(g1, xq, xd1, M, K, threads=oracle.max_threads())
+    assert np.abs(y_ref).max() < 2 ** 24
+    assert np.array_equal(dots.sum(axis=2, dtype=np.int64).astype(np.float64), y_ref)
+    assert np.array_equal(y.astype(np.float64), y_ref)
+
+
 def test_quantize_then_q8q8_end_to_end():
     """GPU quantiser feeding the GPU product equals the oracle chain."""
     M, K, N = 4096, 3584, 16

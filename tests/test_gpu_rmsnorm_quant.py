@@ -96,3 +96,52 @@ def test_rmsnorm_quantize_rejects_bad_eps():
         with pytest.raises(q8().Q8Error) as e:
             q8().q8_rmsnorm_quantize_act(dev(x), dev(np.ones(32, np.float32)), eps, xq, xd, None, 1, 32)
         assert e.value.status == 1
+
+
+def _boundary_margin(x, gamma, eps, r_exact):
+    """For every element, the distance of the exact x_hat / d (fp64: x * r_exact
+    * gamma over amax / 127 of its block) from the nearest half-integer, the
+    points where round-half-away changes the code, and the exact value itself."""
+    N, K = x.shape
+    xh = x.astype(np.float64) * r_exact[:, None] * gamma.astype(np.float64)[None, :]
+    blocks = xh.reshape(N, K // 32, 32)
+    amax = np.abs(blocks).max(axis=2, keepdims=True)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        v = np.where(amax > 0, blocks / (amax / 127.0), 0.0).reshape(N, K)
+    dist = np.abs(np.abs(v) - (np.floor(np.abs(v)) + 0.5))
+    return v, dist
+
+
+@pytest.mark.parametrize("N,K", [(1, 896), (4, 3584), (16, 4864), (2, 18944)])
+def test_rmsnorm_codes_against_exact_r(N, K):
+    """The codes checked against an oracle that does not see the kernel's r:
+    codes taken from r_exact rounded to fp32.  Both sides round x_hat = (x r) g
+    and x_hat / d in fp32, so a code may differ only where the exact x_hat / d
+    sits within the propagated error of a rounding boundary: the kernel's r
+    within (K/256 + 12) 2^-24 of the exact value, plus the fp32 roundings of
+    x r, of the gain product, of amax / 127 and of the division (a few
+    2^-24 each).  Every differing code must be such an element, and they must
+    be rare; the scales may differ only where d = amax / 127 lies that close to
+    a binary16 rounding midpoint."""
+    x = q8gen.activations(170 + N + K, N, K)
+    x[0, :64] *= 50.0
+    g = gain(K, K + 1)
+    eps = 1e-6
+    xq, xd, r = run(x, g, eps)
+    r_exact, _, q_ref, d_ref, d32_ref = oracle.rmsnorm_quantize_act(x, g, eps)  # r = fp32(r_exact)
+    assert np.all(np.abs(r - r_exact) <= r_bound(K) * r_exact)
+    v, dist = _boundary_margin(x, g, eps, r_exact)
+    rel = 2 * r_bound(K) + 8 * 2.0 ** -24
+    near = dist <= rel * np.abs(v) + 2.0 ** -20
+    diff = xq != q_ref
+    assert not np.any(diff & ~near), (
+        f"{int((diff & ~near).sum())} codes differ away from any rounding boundary")
+    assert np.all(np.abs(xq.astype(np.int32) - q_ref.astype(np.int32)) <= 1)
+    assert diff.sum() <= max(2, diff.size // 1000)
+    # binary16 scales: equal unless d sits next to a rounding midpoint
+    dd = xd != d_ref
+    if dd.any():
+        d16 = d_ref.view(np.float16).astype(np.float64)
+        ulp = np.spacing(np.abs(d_ref.view(np.float16))).astype(np.float64)
+        mid_dist = np.abs(np.abs(d32_ref.astype(np.float64) - d16) - ulp / 2)
+        assert np.all(mid_dist[dd] <= (rel + 2.0 ** -23) * np.abs(d32_ref[dd]))
