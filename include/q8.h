@@ -302,11 +302,14 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
  * allocated or freed.
  * The first call on each device looks up the array's device address (with
  * that device current); make that first call before any stream capture.
- * All calls share the one array, which keeps the last call's contents: each
- * call first clears the array's counter region on `stream`
- * (cudaMemsetAsync), then runs the MoE kernel.  Calls that may run at the
- * same time on the GPU (different streams without an ordering between them)
- * race on the array and must not be issued. */
+ * Every argument is checked, as for q8_moe_gemv, before anything is
+ * enqueued.  All calls share the one array, which keeps the last call's
+ * contents: each call first launches a one-warp kernel on `stream` that, once
+ * the work before it on the stream is done, clears the array's counter region,
+ * then the MoE kernel (both as dependent launches, so the MoE kernel still
+ * prefetches its weights early).  Calls that may run at the same time on the
+ * GPU (different streams without an ordering between them) race on the array
+ * and must not be issued. */
 q8_status q8_moe_gemv_noalloc(const void *gate_up_experts, const void *down_experts,
                               const void *shared_gate_up, const void *shared_down,
                               const int32_t *idx, const float *w, const float *x, float *y,
@@ -370,6 +373,24 @@ q8_status q8q8_gemv(const void *W, const int8_t *xq, const uint16_t *xd, float *
  * [N][M][K/32]); bit-exact. */
 q8_status q8q8_block_dots(const void *W, const int8_t *xq, int32_t *dots, int64_t M, int64_t K,
                           int64_t N, q8_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Test aid: the failure-detection protocol                                */
+/* ---------------------------------------------------------------------- */
+
+/* Launches one CTA whose four warps wait, through the same bounded-wait code
+ * as the pipelines' barriers, on a shared-memory barrier that nothing ever
+ * completes, with a limit of `limit_us` microseconds (1 .. 1,000,000) in
+ * place of the pipelines' 2 s.  The first wait to run out sets the timeout
+ * bit (1) of the sticky device error word and the CTA's abort flag; the other
+ * warps leave their waits on seeing the flag, and the kernel returns: no
+ * fault, no hang, and the context stays usable.  out: 2 device int32,
+ * written with the number of warps whose wait succeeded (0) and the abort
+ * flag (1).  q8_read_device_error() then returns Q8_ERR_DEVICE_TIMEOUT with
+ * detail bit 1 set, and clears the word.  Host-side failure handling
+ * (hardened host validation and a device-data trust boundary) follows
+ * "fusedtok 1.3.0", Roadmap 1.2.1; the device-side bound is this library's. */
+q8_status q8_test_wait_timeout(uint32_t limit_us, int32_t *out, q8_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -25,6 +25,7 @@ __all__ = [
     "q8_moe_gemv",
     "q8_moe_gemv_noalloc",
     "q8_quantize_act", "q8_rmsnorm_quantize_act", "q8q8_gemv", "q8q8_block_dots",
+    "q8_test_wait_timeout",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -62,6 +63,7 @@ _SIGS = {
     "q8q8_gemv": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "q8_rmsnorm_quantize_act": (_INT, [_P, _P, ctypes.c_float, _P, _P, _P, _I64, _I64, _P]),
     "q8q8_block_dots": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
+    "q8_test_wait_timeout": (_INT, [ctypes.c_uint32, _P, _P]),
 }
 
 
@@ -243,3 +245,7 @@ def q8q8_gemv(W, xq, xd, y, M, K, N, stream=None):
 
 def q8q8_block_dots(W, xq, dots, M, K, N, stream=None):
     _call("q8q8_block_dots", _ptr(W), _ptr(xq), _ptr(dots), M, K, N, _stream(stream))
+
+
+def q8_test_wait_timeout(limit_us, out, stream=None):
+    _call("q8_test_wait_timeout", int(limit_us), _ptr(out), _stream(stream))

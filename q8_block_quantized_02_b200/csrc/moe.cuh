@@ -1057,4 +1057,15 @@ __global__ void __launch_bounds__(moe_threads(NMAX), 1)
     }
 }
 
+// Zeroes n words of a counter area ahead of a kernel that needs them at zero,
+// as a kernel of the dependent-launch chain: the next kernel may start (and
+// prefetch) at once, and its own dependency wait covers this kernel's stores,
+// which come after this kernel's wait for the grid before it (the previous
+// user of the area).
+__global__ void clear_words_kernel(unsigned *p, int n) {
+    pdl_launch_dependents();
+    pdl_wait();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) p[i] = 0u;
+}
+
 }  // namespace q8

@@ -5,6 +5,8 @@
 // its arguments on the host, picks a launch shape, and enqueues its kernels on
 // the caller's stream with programmatic dependent launch; nothing here
 // allocates, frees or synchronises (q8_read_device_error excepted).
+#include <atomic>
+
 #include "host_common.cuh"
 #include "pack.cuh"
 #include "q8q8.cuh"
@@ -14,6 +16,7 @@
 #include "tile_gemm.cuh"
 #include "moe.cuh"
 #include "kquant.cuh"
+#include "selftest.cuh"
 
 namespace q8 {
 
@@ -614,7 +617,9 @@ static size_t moe_part_bytes(int64_t T, int64_t k, int64_t H, int64_t I, int64_t
 constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;  // 4 MiB
 static __device__ __align__(256) unsigned char g_moe_noalloc_scratch[kNoAllocScratchBytes];
 
-static void *g_moe_noalloc_addr[kMaxDevices];  // device address of the array, per device
+// device address of the array, per device; written once under the mutex
+// (release) and read without it (acquire)
+static std::atomic<void *> g_moe_noalloc_addr[kMaxDevices];
 static std::mutex g_moe_noalloc_mutex;
 
 // The array's name is only a host-side stand-in; the address a kernel can use
@@ -624,19 +629,118 @@ static q8_status moe_noalloc_scratch(void **out) {
     int dev = 0;
     Q8_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice, "device index");
-    if (!g_moe_noalloc_addr[dev]) {
+    void *p = g_moe_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
         std::lock_guard<std::mutex> lock(g_moe_noalloc_mutex);
-        if (!g_moe_noalloc_addr[dev]) {
-            void *p = nullptr;
+        p = g_moe_noalloc_addr[dev].load(std::memory_order_relaxed);
+        if (!p) {
             cudaError_t e = cudaGetSymbolAddress(&p, g_moe_noalloc_scratch);
             if (e != cudaSuccess || p == nullptr)
                 return cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
                                  "cudaGetSymbolAddress(moe scratch)");
-            g_moe_noalloc_addr[dev] = p;
+            g_moe_noalloc_addr[dev].store(p, std::memory_order_release);
         }
     }
-    *out = g_moe_noalloc_addr[dev];
+    *out = p;
     return Q8_OK;
+}
+
+// Host-side checks of q8_moe_gemv's arguments other than its workspace, and
+// its launch plan; nothing is enqueued.
+static q8_status moe_check_args(const void *gate_up_experts, const void *down_experts,
+                                const void *shared_gate_up, const void *shared_down, const int32_t *idx,
+                                const float *w, const float *x, float *y, int64_t T, int64_t E, int64_t top_k,
+                                int64_t H, int64_t I, int64_t I_shared, MoePlan &p) {
+    if (T <= 0 || E <= 0 || top_k <= 0 || top_k > E || H <= 0 || I <= 0 || I_shared < 0)
+        return Q8_ERR_SHAPE;
+    if (H % 32 || I % 32 || I_shared % 32) return Q8_ERR_SHAPE;
+    if (T > kMoeMaxT || top_k > kMoeMaxK || E > kMoeMaxE || H > 65536 || I > 65536 ||
+        I_shared > 65536)
+        return Q8_ERR_UNSUPPORTED;
+    const bool has_shared = shared_gate_up != nullptr || shared_down != nullptr;
+    if (has_shared != (I_shared > 0) || (has_shared && (!shared_gate_up || !shared_down)))
+        return Q8_ERR_INVALID;
+    Q8_CHECK(check_device_ptr(gate_up_experts));
+    Q8_CHECK(check_device_ptr(down_experts));
+    if (has_shared) {
+        Q8_CHECK(check_device_ptr(shared_gate_up));
+        Q8_CHECK(check_device_ptr(shared_down));
+    }
+    Q8_CHECK(check_device_ptr(idx, false));
+    Q8_CHECK(check_device_ptr(w, false));
+    if ((reinterpret_cast<uintptr_t>(idx) | reinterpret_cast<uintptr_t>(w)) & 3u) return Q8_ERR_ALIGN;
+    Q8_CHECK(check_device_ptr(x));
+    Q8_CHECK(check_device_ptr(y));
+    const DeviceInfo *dev = nullptr;
+    Q8_CHECK(device_info(&dev));
+    if (!plan_moe(T, dev->max_smem_optin, p)) return Q8_ERR_UNSUPPORTED;
+    return Q8_OK;
+}
+
+// Encodes the tensor maps and launches the MoE kernel (arguments checked).
+static q8_status moe_launch(MoePlan &p, const void *gate_up_experts, const void *down_experts,
+                            const void *shared_gate_up, const void *shared_down, const int32_t *idx,
+                            const float *w, const float *x, float *y, int64_t T, int64_t E, int64_t top_k,
+                            int64_t H, int64_t I, int64_t I_shared, void *workspace, cudaStream_t stream) {
+    const DeviceInfo *dev = nullptr;
+    Q8_CHECK(device_info(&dev));
+    const bool has_shared = shared_gate_up != nullptr;
+    MoeArgs &a = p.a;
+    const int64_t Ish = has_shared ? I_shared : 0;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    a.T = (int)T; a.E = (int)E; a.k = (int)top_k; a.H = (int)H; a.I = (int)I; a.Is = (int)Ish;
+    moe_shared_chunks(I, Ish, a.nsplit, a.cc);
+    a.idx = idx;
+    a.w = w;
+    a.y = y;
+    a.ctr = reinterpret_cast<unsigned *>(ws);
+    a.hbuf = reinterpret_cast<float *>(ws + moe_ctr_bytes(H));
+    a.hsh = reinterpret_cast<float *>(ws + moe_ctr_bytes(H) + moe_hbuf_bytes(T, top_k, I));
+    a.part = reinterpret_cast<float *>(ws + moe_ctr_bytes(H) + moe_hbuf_bytes(T, top_k, I) +
+                                       moe_hsh_bytes(T, I_shared));
+
+    // Weight maps: [16-byte column][8 rows x 16 B] q boxes and [block][8 rows]
+    // fp16 scale boxes of 1, 2, 4 or 8 consecutive packed groups (the tile
+    // kernels' layout).  Activation maps: [row][column][16 fp32], one row per
+    // box, or all T rows for the shared expert's segment.
+    MoeMaps m;
+    const uint8_t *gu = static_cast<const uint8_t *>(gate_up_experts);
+    const uint8_t *dn = static_cast<const uint8_t *>(down_experts);
+    // weight maps of every box depth (see moe.cuh): [phase][routed|shared][q|scales][depth]
+    auto weight_maps = [&](CUtensorMap(&w)[2][kMoeDepths], const uint8_t *base, int64_t K, int64_t groups)
+        -> q8_status {
+        const uint64_t gs = (uint64_t)kGroupBytesPerBlock * (K / 32);
+        for (int d = 0; d < kMoeDepths; ++d) {
+            Q8_CHECK(make_map_3d(&w[0][d], CU_TENSOR_MAP_DATA_TYPE_UINT8, base, kColBytes, K / 16, groups,
+                                 kColBytes, gs, kColBytes, kMoeCS, 1u << d, true));
+            Q8_CHECK(make_map_3d(&w[1][d], CU_TENSOR_MAP_DATA_TYPE_UINT16, base + 256 * (K / 32), 8, K / 32,
+                                 groups, 16, gs, 8, kMoeCS / 2, 1u << d, true));
+        }
+        return Q8_OK;
+    };
+    Q8_CHECK(weight_maps(m.w[0][0], gu, H, E * (2 * I / 8)));
+    Q8_CHECK(weight_maps(m.w[1][0], dn, I, E * (H / 8)));
+    Q8_CHECK(make_map_3d(&m.x1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, H / 16, T, 64, (uint64_t)H * 4, 16, kMoeCS,
+                         1, false));
+    Q8_CHECK(make_map_3d(&m.x1s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, H / 16, T, 64, (uint64_t)H * 4, 16, kMoeCS,
+                         (uint32_t)T, false));
+    Q8_CHECK(make_map_3d(&m.h2r, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.hbuf, 16, I / 16, T * top_k, 64,
+                         (uint64_t)I * 4, 16, kMoeCS, 1, false));
+    if (has_shared) {
+        const uint8_t *sgu = static_cast<const uint8_t *>(shared_gate_up);
+        const uint8_t *sdn = static_cast<const uint8_t *>(shared_down);
+        Q8_CHECK(weight_maps(m.w[0][1], sgu, H, 2 * Ish / 8));
+        Q8_CHECK(weight_maps(m.w[1][1], sdn, Ish, H / 8));
+        Q8_CHECK(make_map_3d(&m.h2s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.hsh, 16, Ish / 16, T, 64,
+                             (uint64_t)Ish * 4, 16, kMoeCS, (uint32_t)T, false));
+    } else {
+        for (int ph = 0; ph < 2; ++ph)
+            for (int qd = 0; qd < 2; ++qd)
+                for (int d = 0; d < kMoeDepths; ++d) m.w[ph][1][qd][d] = m.w[ph][0][qd][d];
+        m.h2s = m.h2r;
+    }
+    return launch_pdl(moe_kernel_for(nmax_for(T)), dim3((unsigned)dev->sms), dim3(moe_threads(nmax_for(T))), p.smem,
+                      stream, "q8_moe_gemv launch", m, a);
 }
 
 template <int FMT>
@@ -891,88 +995,13 @@ q8_status q8_moe_gemv(const void *gate_up_experts, const void *down_experts,
                       const int32_t *idx, const float *w, const float *x, float *y, int64_t T,
                       int64_t E, int64_t top_k, int64_t H, int64_t I, int64_t I_shared,
                       void *workspace, size_t workspace_bytes, q8_stream_t stream) {
-    if (T <= 0 || E <= 0 || top_k <= 0 || top_k > E || H <= 0 || I <= 0 || I_shared < 0)
-        return Q8_ERR_SHAPE;
-    if (H % 32 || I % 32 || I_shared % 32) return Q8_ERR_SHAPE;
-    if (T > kMoeMaxT || top_k > kMoeMaxK || E > kMoeMaxE || H > 65536 || I > 65536 ||
-        I_shared > 65536)
-        return Q8_ERR_UNSUPPORTED;
-    const bool has_shared = shared_gate_up != nullptr || shared_down != nullptr;
-    if (has_shared != (I_shared > 0) || (has_shared && (!shared_gate_up || !shared_down)))
-        return Q8_ERR_INVALID;
-    Q8_CHECK(check_device_ptr(gate_up_experts));
-    Q8_CHECK(check_device_ptr(down_experts));
-    if (has_shared) {
-        Q8_CHECK(check_device_ptr(shared_gate_up));
-        Q8_CHECK(check_device_ptr(shared_down));
-    }
-    Q8_CHECK(check_device_ptr(idx, false));
-    Q8_CHECK(check_device_ptr(w, false));
-    if ((reinterpret_cast<uintptr_t>(idx) | reinterpret_cast<uintptr_t>(w)) & 3u) return Q8_ERR_ALIGN;
-    Q8_CHECK(check_device_ptr(x));
-    Q8_CHECK(check_device_ptr(y));
+    MoePlan p;
+    Q8_CHECK(moe_check_args(gate_up_experts, down_experts, shared_gate_up, shared_down, idx, w, x, y, T, E,
+                            top_k, H, I, I_shared, p));
     Q8_CHECK(check_device_ptr(workspace));
     if (workspace_bytes < q8_moe_workspace_bytes(T, E, top_k, H, I, I_shared)) return Q8_ERR_SHAPE;
-    const DeviceInfo *dev = nullptr;
-    Q8_CHECK(device_info(&dev));
-    MoePlan p;
-    if (!plan_moe(T, dev->max_smem_optin, p)) return Q8_ERR_UNSUPPORTED;
-    MoeArgs &a = p.a;
-    const int64_t Ish = has_shared ? I_shared : 0;
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    a.T = (int)T; a.E = (int)E; a.k = (int)top_k; a.H = (int)H; a.I = (int)I; a.Is = (int)Ish;
-    moe_shared_chunks(I, Ish, a.nsplit, a.cc);
-    a.idx = idx;
-    a.w = w;
-    a.y = y;
-    a.ctr = reinterpret_cast<unsigned *>(ws);
-    a.hbuf = reinterpret_cast<float *>(ws + moe_ctr_bytes(H));
-    a.hsh = reinterpret_cast<float *>(ws + moe_ctr_bytes(H) + moe_hbuf_bytes(T, top_k, I));
-    a.part = reinterpret_cast<float *>(ws + moe_ctr_bytes(H) + moe_hbuf_bytes(T, top_k, I) +
-                                       moe_hsh_bytes(T, I_shared));
-
-    // Weight maps: [16-byte column][8 rows x 16 B] q boxes and [block][8 rows]
-    // fp16 scale boxes of 1, 2, 4 or 8 consecutive packed groups (the tile
-    // kernels' layout).  Activation maps: [row][column][16 fp32], one row per
-    // box, or all T rows for the shared expert's segment.
-    MoeMaps m;
-    const uint8_t *gu = static_cast<const uint8_t *>(gate_up_experts);
-    const uint8_t *dn = static_cast<const uint8_t *>(down_experts);
-    // weight maps of every box depth (see moe.cuh): [phase][routed|shared][q|scales][depth]
-    auto weight_maps = [&](CUtensorMap(&w)[2][kMoeDepths], const uint8_t *base, int64_t K, int64_t groups)
-        -> q8_status {
-        const uint64_t gs = (uint64_t)kGroupBytesPerBlock * (K / 32);
-        for (int d = 0; d < kMoeDepths; ++d) {
-            Q8_CHECK(make_map_3d(&w[0][d], CU_TENSOR_MAP_DATA_TYPE_UINT8, base, kColBytes, K / 16, groups,
-                                 kColBytes, gs, kColBytes, kMoeCS, 1u << d, true));
-            Q8_CHECK(make_map_3d(&w[1][d], CU_TENSOR_MAP_DATA_TYPE_UINT16, base + 256 * (K / 32), 8, K / 32,
-                                 groups, 16, gs, 8, kMoeCS / 2, 1u << d, true));
-        }
-        return Q8_OK;
-    };
-    Q8_CHECK(weight_maps(m.w[0][0], gu, H, E * (2 * I / 8)));
-    Q8_CHECK(weight_maps(m.w[1][0], dn, I, E * (H / 8)));
-    Q8_CHECK(make_map_3d(&m.x1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, H / 16, T, 64, (uint64_t)H * 4, 16, kMoeCS,
-                         1, false));
-    Q8_CHECK(make_map_3d(&m.x1s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x, 16, H / 16, T, 64, (uint64_t)H * 4, 16, kMoeCS,
-                         (uint32_t)T, false));
-    Q8_CHECK(make_map_3d(&m.h2r, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.hbuf, 16, I / 16, T * top_k, 64,
-                         (uint64_t)I * 4, 16, kMoeCS, 1, false));
-    if (has_shared) {
-        const uint8_t *sgu = static_cast<const uint8_t *>(shared_gate_up);
-        const uint8_t *sdn = static_cast<const uint8_t *>(shared_down);
-        Q8_CHECK(weight_maps(m.w[0][1], sgu, H, 2 * Ish / 8));
-        Q8_CHECK(weight_maps(m.w[1][1], sdn, Ish, H / 8));
-        Q8_CHECK(make_map_3d(&m.h2s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.hsh, 16, Ish / 16, T, 64,
-                             (uint64_t)Ish * 4, 16, kMoeCS, (uint32_t)T, false));
-    } else {
-        for (int ph = 0; ph < 2; ++ph)
-            for (int qd = 0; qd < 2; ++qd)
-                for (int d = 0; d < kMoeDepths; ++d) m.w[ph][1][qd][d] = m.w[ph][0][qd][d];
-        m.h2s = m.h2r;
-    }
-    return launch_pdl(moe_kernel_for(nmax_for(T)), dim3((unsigned)dev->sms), dim3(moe_threads(nmax_for(T))), p.smem,
-                      (cudaStream_t)stream, "q8_moe_gemv launch", m, a);
+    return moe_launch(p, gate_up_experts, down_experts, shared_gate_up, shared_down, idx, w, x, y, T, E, top_k,
+                      H, I, I_shared, workspace, (cudaStream_t)stream);
 }
 
 q8_status q8_moe_gemv_noalloc(const void *gate_up_experts, const void *down_experts,
@@ -989,14 +1018,29 @@ q8_status q8_moe_gemv_noalloc(const void *gate_up_experts, const void *down_expe
                  need, kNoAllocScratchBytes);
         return Q8_ERR_UNSUPPORTED;
     }
+    // every argument is checked before anything is enqueued
+    MoePlan p;
+    Q8_CHECK(moe_check_args(gate_up_experts, down_experts, shared_gate_up, shared_down, idx, w, x, y, T, E,
+                            top_k, H, I, I_shared, p));
     void *scratch = nullptr;
     Q8_CHECK(moe_noalloc_scratch(&scratch));
     // The array keeps whatever the previous call left in it; the MoE kernel
-    // needs its counters at zero when it starts, so clear them on the stream
-    // first (a memset node, no allocation).
-    Q8_CUDA_TRY(cudaMemsetAsync(scratch, 0, moe_ctr_bytes(H), (cudaStream_t)stream));
-    return q8_moe_gemv(gate_up_experts, down_experts, shared_gate_up, shared_down, idx, w, x, y, T,
-                       E, top_k, H, I, I_shared, scratch, need, stream);
+    // needs its counters at zero when its dependency wait returns.  A one-warp
+    // kernel of the dependent-launch chain clears them (a memset node there
+    // would stop the MoE kernel from starting early and prefetching weights).
+    const int words = (int)(moe_ctr_bytes(H) / 4);
+    Q8_CHECK(launch_pdl(clear_words_kernel, dim3(1), dim3(32), 0, (cudaStream_t)stream,
+                        "q8_moe_gemv_noalloc clear launch", static_cast<unsigned *>(scratch), words));
+    return moe_launch(p, gate_up_experts, down_experts, shared_gate_up, shared_down, idx, w, x, y, T, E, top_k,
+                      H, I, I_shared, scratch, (cudaStream_t)stream);
+}
+
+q8_status q8_test_wait_timeout(uint32_t limit_us, int32_t *out, q8_stream_t stream) {
+    if (limit_us == 0 || limit_us > 1000000u) return Q8_ERR_UNSUPPORTED;
+    Q8_CHECK(check_device_ptr(out, false));
+    if (reinterpret_cast<uintptr_t>(out) & 3u) return Q8_ERR_ALIGN;
+    return launch_pdl(wait_timeout_kernel, dim3(1), dim3(kSelftestThreads), 0, (cudaStream_t)stream,
+                      "q8_test_wait_timeout launch", (uint64_t)limit_us * 1000ull, reinterpret_cast<int *>(out));
 }
 
 }  // extern "C"

@@ -104,14 +104,16 @@ constexpr uint32_t kWaitHintNs = 20000;
 // raises *abort) when the wait runs past kWaitLimitNs; returns false at once
 // when *abort is already raised, so that every thread of a CTA leaves a broken
 // pipeline quickly and still reaches the CTA's remaining barriers.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort) {
+// (`limit_ns` is the wait limit; only the wait self-test passes a shorter one.)
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort && *abort) return false;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
         if (abort && *abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             record_error(kErrWaitTimeout);
             if (abort) *abort = 1;
             return false;
@@ -122,9 +124,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // mbar_wait for a whole warp: lane 0 alone polls the barrier (32 lanes polling
 // one barrier serialise in the shared-memory pipe), then __syncwarp orders its
 // acquire before every lane's reads of the guarded data.  Warp-uniform result.
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort) {
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort,
+                                               uint64_t limit_ns = kWaitLimitNs) {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, limit_ns) ? 1 : 0;
     __syncwarp();
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }

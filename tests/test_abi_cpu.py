@@ -198,6 +198,12 @@ def test_host_validation_runs_before_any_device_work(lib):
     msg = lib.q8_last_cuda_error
     msg.restype = ctypes.c_char_p
     assert b"4194304" in msg()
+    # small valid sizes with null buffers: rejected by the argument checks,
+    # before the scratch address is looked up or anything is enqueued
+    assert noalloc(n, n, n, n, n, n, n, n, 1, 60, 4, 2048, 1408, 5632, n) == 1
+    assert noalloc(n, n, n, n, n, n, n, n, 1, 60, 4, 2048, 1408, 0, n) == 1
+    assert noalloc(n, n, n, n, n, n, n, n, 1, 60, 4, 2000, 1408, 0, n) == 2          # H % 32
+    assert noalloc(n, n, n, n, n, n, n, n, 17, 60, 4, 2048, 1408, 0, n) == 5         # T > 16
     pack = fn("q8_pack_weights", P, I64, I64, P, P)
     assert pack(n, 8, 40, n, n) == 2
     init = fn("q8_moe_workspace_init", P, ctypes.c_size_t, P)
