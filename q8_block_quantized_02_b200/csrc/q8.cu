@@ -14,6 +14,7 @@
 #include "f32_mma.cuh"
 #include "route.cuh"
 #include "tile_gemm.cuh"
+#include "resident.cuh"
 #include "moe.cuh"
 #include "kquant.cuh"
 #include "selftest.cuh"
@@ -189,11 +190,10 @@ static TilePlan plan_tile(int64_t units, int64_t C, int64_t N, int mode, int sms
 // resident kernel: small matrices whose CTA-share of weights fits in shared
 // memory (see tile_gemm.cuh)
 // ---------------------------------------------------------------------------
-using ResidentKernel = void (*)(CUtensorMap, CUtensorMap, const float *, TileArgs);
+using ResidentKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, const float *, TileArgs);
 
-// N = 1 only: a CTA of this kernel leaves most of the SM's registers to the
-// next kernel on the stream (wider N would take them all).  One instance per
-// row-group count, so the column step needs no per-group branch.
+// N = 1 only.  One instance per row-group count, so the column step needs no
+// per-group branch.
 template <int MODE>
 static ResidentKernel resident_kernel_mode(int tgm) {
     switch (tgm) {
@@ -210,8 +210,24 @@ static ResidentKernel resident_kernel_mode(int tgm) {
 static ResidentKernel resident_kernel_for(int mode, int tgm) {
     return mode == kModeSwiGLU ? resident_kernel_mode<kModeSwiGLU>(tgm) : resident_kernel_mode<kModeF32>(tgm);
 }
-static int resident_red_floats(int mode) {
-    return mode == kModeSwiGLU ? res_red_floats<1, kModeSwiGLU>() : res_red_floats<1, kModeF32>();
+template <int MODE>
+static int resident_red_floats_mode(int tgm) {
+    switch (tgm) {
+        case 1: return res_red_floats<1, MODE, 1>();
+        case 2: return res_red_floats<1, MODE, 2>();
+        case 3: return res_red_floats<1, MODE, 3>();
+        case 4: return res_red_floats<1, MODE, 4>();
+        case 5: return res_red_floats<1, MODE, 5>();
+        case 6: return res_red_floats<1, MODE, 6>();
+        case 7: return res_red_floats<1, MODE, 7>();
+        default: return res_red_floats<1, MODE, 8>();
+    }
+}
+static int resident_red_floats(int mode, int tgm) {
+    return mode == kModeSwiGLU ? resident_red_floats_mode<kModeSwiGLU>(tgm) : resident_red_floats_mode<kModeF32>(tgm);
+}
+static int resident_threads(int mode, int tgm) {
+    return 32 * (mode == kModeF32 && tgm == 1 ? res_warps<kModeF32, 1>() : res_warps<kModeSwiGLU, 2>());
 }
 
 static cudaError_t setup_resident_kernels(int max_smem) {
@@ -267,11 +283,11 @@ static bool plan_resident(int64_t units, int64_t C, int64_t N, int mode, int sms
     a.d_half = (uint32_t)(upc * a.d_box);
     a.x_off = a.d_off + (uint32_t)(halves * a.d_half);
     a.stage_bytes = (uint32_t)round_up(a.x_off + a.x_box, 128);
-    const int64_t smem = (int64_t)a.stage_bytes + (int64_t)resident_red_floats(mode) * 4 + 16;
+    const int64_t smem = (int64_t)a.stage_bytes + (int64_t)resident_red_floats(mode, (int)upc) * 4 + 16;
     if (smem > kResidentSmemBudget) return false;
     if (halves * upc * (int64_t)(a.q_box + a.d_box) >= (1 << 20)) return false;  // mbarrier tx count
     p.grid = (int)grid;
-    p.threads = kResThreads;
+    p.threads = resident_threads(mode, (int)upc);
     p.wide = false;
     p.smem = (size_t)smem;
     *out = p;
@@ -292,13 +308,21 @@ static q8_status run_resident(const TilePlan &plan, const void *W, const float *
     a.up_group0 = swiglu ? a.units : 0;
     const uint64_t gstride = (uint64_t)kGroupBytesPerBlock * B;
     const uint8_t *dbase = static_cast<const uint8_t *>(W) + 256 * B;
-    CUtensorMap tq, td;
+    // one chunk: maps whose box depth is the CTA's row-group count (TG, or
+    // TG - 1 on the CTAs holding one fewer); several chunks: depth 1
+    const uint32_t depth = a.nchunks == 1 ? (uint32_t)a.TG : 1u;
+    const uint32_t depth1 = a.nchunks == 1 && a.TG > 1 ? (uint32_t)a.TG - 1 : depth;
+    CUtensorMap tq, td, tq1, td1;
     Q8_CHECK(make_map_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, kColBytes, C, total_groups, kColBytes,
-                         gstride, kColBytes, a.CB, 1, true));
+                         gstride, kColBytes, a.CB, depth, true));
     Q8_CHECK(make_map_3d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT16, dbase, 8, B, total_groups, 16, gstride, 8,
-                         a.CB / 2, 1, true));
+                         a.CB / 2, depth, true));
+    Q8_CHECK(make_map_3d(&tq1, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, kColBytes, C, total_groups, kColBytes,
+                         gstride, kColBytes, a.CB, depth1, true));
+    Q8_CHECK(make_map_3d(&td1, CU_TENSOR_MAP_DATA_TYPE_UINT16, dbase, 8, B, total_groups, 16, gstride, 8,
+                         a.CB / 2, depth1, true));
     return launch_pdl(resident_kernel_for(mode, a.TG), dim3(p.grid), dim3(p.threads), p.smem, stream,
-                      swiglu ? "q8_gate_up_swiglu launch" : "q8_gemv launch", tq, td, x, a);
+                      swiglu ? "q8_gate_up_swiglu launch" : "q8_gemv launch", tq, td, tq1, td1, x, a);
 }
 
 static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_out, int64_t K,

@@ -1,8 +1,8 @@
 """GPU parity of the resident GEMV kernel (small matrices at N = 1) against
-the fp64 oracle, across its planning regimes: one row group per CTA (each
-thread owns whole columns, up to 512 of them in all), several row groups per
-CTA (column-owner lanes), the SwiGLU pair, ragged last groups, and shapes too
-large for it (the column kernel takes them).  Also a
+the fp64 oracle, across its planning regimes: one row group per CTA, several
+row groups per CTA (CTAs holding TGM or TGM - 1 of them), one or two column
+chunks, the SwiGLU pair, ragged last groups, and shapes too large for it (the
+column kernel takes them).  Also a
 chain of dependent launches on one stream, as a decode step issues them."""
 from __future__ import annotations
 
@@ -17,13 +17,14 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("M,K", [
     (1152, 896),    # 144 groups on 144 CTAs, 56 columns
-    (896, 4864),    # 304 columns: some threads own two
-    (100, 8192),    # 512 columns: every thread owns two (too large: column kernel)
+    (896, 4864),    # 304 columns in two chunks of 160 (the second one zero-filled past K)
+    (100, 8192),    # 512 columns (too large: column kernel)
     (100, 6144),    # 13 groups, 384 columns
     (1157, 896),    # ragged last group (5 rows)
     (2000, 896),    # 250 groups: two per CTA on most CTAs
     (6000, 1408),   # six groups per CTA
     (9000, 896),    # eight groups per CTA
+    (1200, 4608),   # two chunks of 144 columns, one or two groups per CTA
     (9000, 4864),   # too large for shared memory: column kernel
 ])
 def test_resident_gemv_matches_oracle(M, K):
@@ -36,8 +37,9 @@ def test_resident_gemv_matches_oracle(M, K):
 @pytest.mark.parametrize("I,K", [
     (4864, 896),    # 608 gate groups: four or five per CTA
     (1408, 2048),   # two groups per CTA, 128 columns
-    (104, 4864),    # one gate group per CTA, 304 columns
+    (104, 4864),    # one gate group per CTA, 304 columns (column kernel: over the shared-memory budget)
     (2400, 1024),   # three groups per CTA
+    (160, 4608),    # two chunks of 144 columns, gate and up
     (9000, 896),    # too large for shared memory: column kernel
 ])
 def test_resident_swiglu_matches_oracle(I, K):
