@@ -12,7 +12,10 @@ weights are larger than L2, so no flush is needed between steps.
 Reports one JSON line (see --help): tokens/s over all GPUs, the HBM GB/s the
 step achieves (34 bytes per 32 weights), the roofline of the dominant kernel,
 an end-to-end figure with host copies, clocks seen during the timed region,
-and the CPU oracle timed on the host as a baseline.
+the CPU oracle timed on the host as a baseline (all cores and one thread),
+and, under "configs", the device time per call of the other workloads (the
+single 1152x896 GEMV, the 7B-class products at N = 1..16, the Qwen1.5-MoE
+block at T = 1 and 8, the Q8 x Q8 sweep) with the oracle's time beside each.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
 
@@ -73,6 +76,23 @@ def measured_hbm_peak():
 
 def algorithmic_bytes(M, K):
     return M * K * 34 // 32
+
+
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "resident_gemv_decode_chain_qwen05b.md")
+
+
+def measured_traffic():
+    """DRAM bytes (read + write) per launch of the dominant kernel, from the
+    committed ncu summary of the same kernel in the same decode chain (the
+    line `traffic_bytes_per_launch: <n>`); None when there is none."""
+    try:
+        with open(TRAFFIC_PROFILE) as f:
+            for line in f:
+                if line.strip().startswith("traffic_bytes_per_launch:"):
+                    return int(line.split(":", 1)[1].strip().split()[0])
+    except (OSError, ValueError):
+        pass
+    return None
 
 
 # ---------------------------------------------------------------------------
@@ -146,6 +166,200 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "samples": len(sm),
                 "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# the other workloads: one product per call, device time per call
+# ---------------------------------------------------------------------------
+
+def _graph_time_us(torch, stream, calls, replays=5):
+    """Capture `calls` (a list of zero-argument launches on `stream`) in one
+    CUDA graph, replay it, and return device microseconds per call (CUDA
+    events on the launch stream around `replays` replays, after 2 untimed)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for c in calls:
+            c()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(replays):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (replays * len(calls))
+    del g
+    return us
+
+
+def gpu_configs(q8, torch, dev, stream):
+    """Device time per call of the single GEMV (1152x896, seed 0), the 7B-class
+    small-batch products (N = 1, 2, 4, 8, 16), the Qwen1.5-MoE block (T = 1, 8)
+    and the Q8 x Q8 sweep (M = 4096, K in {896, 3584, 4864, 18944}, N in {1,
+    16}).  Calls walk distinct packed copies of each matrix covering several
+    times the L2 (the same bytes, so only the cache behaviour differs), or
+    distinct routings for the MoE block, so every call streams its weights
+    from HBM.  Weight bytes are 34 per 32 weights."""
+    import numpy as np
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    out = {}
+
+    def packed_copies(g, M, K, min_bytes):
+        nbytes = q8.q8_packed_bytes(M, K)
+        n = max(1, int(np.ceil(min_bytes / nbytes)))
+        src = torch.from_numpy(g).to(dev)
+        ps = []
+        for _ in range(n):
+            p = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+            q8.q8_pack_weights(src, M, K, p, stream=stream)
+            ps.append(p)
+        del src
+        return ps
+
+    # single GEMV at the exact seed, rotated over >= 4 x L2 of copies
+    M, K = 1152, 896
+    g, x = q8gen.q8_matrix(0, M, K, 1)
+    ps = packed_copies(g, M, K, 4 * l2)
+    xd = torch.from_numpy(x).to(dev)
+    y = torch.empty((1, M), dtype=torch.float32, device=dev)
+    us = _graph_time_us(torch, stream, [lambda p=p: q8.q8_gemv(p, xd, y, M, K, 1, stream=stream) for p in ps])
+    out["gemv_1152x896_n1_seed0"] = {"us_per_call": round(us, 3),
+                                     "weight_GBps": round(algorithmic_bytes(M, K) / us / 1e3, 1),
+                                     "rotation": f"{len(ps)} packed copies ({len(ps) * q8.q8_packed_bytes(M, K) >> 20} MiB)"}
+    del ps
+
+    # 7B-class small-batch products
+    for spec in q8gen.small_batch_matrices_7b():
+        g, _ = q8gen.q8_matrix(spec.seed, spec.M, spec.K)
+        ps = packed_copies(g, spec.M, spec.K, 2 * l2)
+        rows = spec.M // 2 if spec.swiglu else spec.M
+        res = {}
+        for N in (1, 2, 4, 8, 16):
+            xd = torch.from_numpy(q8gen.activations(100 + N, N, spec.K)).to(dev)
+            y = torch.empty((N, rows), dtype=torch.float32, device=dev)
+            if spec.swiglu:
+                calls = [lambda p=p: q8.q8_gate_up_swiglu(p, xd, y, rows, spec.K, N, stream=stream) for p in ps]
+            else:
+                calls = [lambda p=p: q8.q8_gemv(p, xd, y, spec.M, spec.K, N, stream=stream) for p in ps]
+            us = _graph_time_us(torch, stream, calls * max(1, 4 // len(ps)))
+            res[f"N={N}"] = {"us_per_call": round(us, 2),
+                             "weight_GBps": round(algorithmic_bytes(spec.M, spec.K) / us / 1e3, 1)}
+        key = f"7b_{spec.name}_{spec.M}x{spec.K}" + ("_swiglu" if spec.swiglu else "")
+        out[key] = res
+        del ps
+
+    # Qwen1.5-MoE block: 60 experts + shared expert, top-4, cycling 16 routings
+    E, H, I, Is, k = 60, 2048, 1408, 5632, 4
+
+    def stack(seed0, n, Mx, Kx):
+        one = q8.q8_packed_bytes(Mx, Kx)
+        buf = torch.empty(n * one, dtype=torch.uint8, device=dev)
+        for e in range(n):
+            ge, _ = q8gen.q8_matrix(seed0 + e, Mx, Kx)
+            q8.q8_pack_weights(torch.from_numpy(ge).to(dev), Mx, Kx, buf[e * one:(e + 1) * one], stream=stream)
+        return buf
+
+    p_gu, p_dn = stack(0, E, 2 * I, H), stack(1000, E, H, I)
+    p_sgu, p_sdn = stack(E, 1, 2 * Is, H), stack(1000 + E, 1, H, Is)
+    per_expert = (2 * I * H + H * I) * 34 // 32
+    shared = (2 * Is * H + H * Is) * 34 // 32
+    for T in (1, 8):
+        R = 16
+        idx = torch.empty((R, T, k), dtype=torch.int32, device=dev)
+        w = torch.empty((R, T, k), dtype=torch.float32, device=dev)
+        for r in range(R):
+            lg = torch.from_numpy(q8gen.logits(61 + 100 * T + r, T, E)).to(dev)
+            q8.q8_moe_route(lg, T, E, k, 0, idx[r], w[r], stream=stream)
+        xd = torch.from_numpy(q8gen.activations(61, T, H)).to(dev)
+        y = torch.empty((T, H), dtype=torch.float32, device=dev)
+        ws_bytes = q8.q8_moe_workspace_bytes(T, E, k, H, I, Is)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        q8.q8_moe_workspace_init(ws, ws_bytes, stream=stream)
+        calls = [lambda r=r: q8.q8_moe_gemv(p_gu, p_dn, p_sgu, p_sdn, idx[r], w[r], xd, y, T, E, k, H, I, Is,
+                                            ws, ws_bytes, stream=stream) for r in range(R)]
+        us = _graph_time_us(torch, stream, calls)
+        picks = idx.cpu().numpy()
+        mean_bytes = float(np.mean([len(np.unique(picks[r])) for r in range(R)])) * per_expert + shared
+        out[f"moe_qwen1.5_a2.7b_T{T}"] = {"us_per_call": round(us, 2), "weight_MB_per_call": round(mean_bytes / 1e6, 2),
+                                          "weight_GBps": round(mean_bytes / us / 1e3, 1),
+                                          "rotation": f"{R} routings of N(0,1) logits, cycled"}
+    del p_gu, p_dn, p_sgu, p_sdn
+
+    # Q8 x Q8: quantise the activations (timed on its own), then the integer product
+    M = 4096
+    q8q8 = {}
+    for K in (896, 3584, 4864, 18944):
+        g, _ = q8gen.q8_matrix(K, M, K)
+        ps = packed_copies(g, M, K, 4 * l2)
+        for N in (1, 16):
+            xf = torch.from_numpy(q8gen.activations(K + N, N, K)).to(dev)
+            xq = torch.empty((N, K), dtype=torch.int8, device=dev)
+            xd = torch.empty((N, K // 32), dtype=torch.int16, device=dev)
+            y = torch.empty((N, M), dtype=torch.float32, device=dev)
+            us_q = _graph_time_us(torch, stream, [lambda: q8.q8_quantize_act(xf, xq, xd, N, K, stream=stream)] * 20)
+            us = _graph_time_us(torch, stream, [lambda p=p: q8.q8q8_gemv(p, xq, xd, y, M, K, N, stream=stream)
+                                                for p in ps])
+            q8q8[f"K={K},N={N}"] = {"us_per_call": round(us, 3), "quantize_us": round(us_q, 3),
+                                    "weight_GBps": round(algorithmic_bytes(M, K) / us / 1e3, 1)}
+        del ps
+    out["q8q8_m4096"] = q8q8
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def oracle_configs(threads):
+    """The fp64 CPU oracle on the same workloads (all host cores, OpenMP over
+    output rows), each on a bounded sample: the whole single GEMV and MoE
+    block; 128 rows of the large matrices, scaled to the full row count."""
+    import oracle
+    out = {}
+
+    def timed(fn, min_s=0.3):
+        n, t0 = 0, time.perf_counter()
+        while True:
+            fn()
+            n += 1
+            dt = time.perf_counter() - t0
+            if dt >= min_s:
+                return dt / n * 1e6
+
+    g, x = q8gen.q8_matrix(0, 1152, 896, 1)
+    out["gemv_1152x896_n1_seed0"] = {"oracle_us_per_call": round(timed(lambda: oracle.gemv(g, x, 1152, 896, threads=threads)), 1),
+                                     "oracle_sample": "whole matrix"}
+    S = 128
+    for spec in q8gen.small_batch_matrices_7b():
+        g, _ = q8gen.q8_matrix(spec.seed, S if not spec.swiglu else 2 * S, spec.K)
+        res = {}
+        for N in (1, 16):
+            xs = q8gen.activations(100 + N, N, spec.K)
+            if spec.swiglu:
+                us = timed(lambda: oracle.gate_up_swiglu(g, xs, S, spec.K, threads=threads)) * (spec.M // 2) / S
+            else:
+                us = timed(lambda: oracle.gemv(g, xs, S, spec.K, threads=threads)) * spec.M / S
+            res[f"N={N}"] = round(us, 1)
+        key = f"7b_{spec.name}_{spec.M}x{spec.K}" + ("_swiglu" if spec.swiglu else "")
+        out[key] = {"oracle_us_per_call": res, "oracle_sample": f"{S} output rows, scaled to {spec.M // (2 if spec.swiglu else 1)}"}
+    E, H, I, Is, k = 60, 2048, 1408, 5632, 4
+    gu, dn, sgu, sdn = q8gen.moe_weights(E, H, I, Is)
+    for T in (1, 8):
+        lg = q8gen.logits(61 + 100 * T, T, E)
+        idx, w = oracle.route(lg, k)
+        xs = q8gen.activations(61, T, H)
+        us = timed(lambda: oracle.moe(gu, dn, sgu, sdn, idx, w, xs, H, I, Is, threads=threads), 0.5)
+        out[f"moe_qwen1.5_a2.7b_T{T}"] = {"oracle_us_per_call": round(us, 1), "oracle_sample": "whole block"}
+    q = {}
+    for K in (896, 3584, 4864, 18944):
+        g, _ = q8gen.q8_matrix(K, S, K)
+        for N in (1, 16):
+            xq, xd, _ = oracle.quantize_act(q8gen.activations(K + N, N, K))
+            q[f"K={K},N={N}"] = round(timed(lambda: oracle.q8q8(g, xq, xd, S, K, want_dots=False, threads=threads))
+                                      * 4096 / S, 1)
+    out["q8q8_m4096"] = {"oracle_us_per_call": q, "oracle_sample": f"{S} output rows, scaled to 4096"}
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -336,13 +550,26 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
 
-    # ---- CPU oracle baseline (rank 0, single GPU only) ----
-    cpu = None
+    # ---- the other workloads, one product per call (single GPU only) ----
+    configs = None
+    if world == 1 and not args.no_configs:
+        with torch.cuda.stream(stream):
+            configs = gpu_configs(q8, torch, dev, stream)
+
+    # ---- CPU oracle baseline (rank 0, single GPU only): all host cores and
+    # one thread, the row split across threads of "Lumen v0.3.0" Phase 7.J ----
+    cpu = cpu1 = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r, tokens, dt, threads = oracle_decode_tokens(host_weights, host_x, target_s=args.cpu_seconds)
         cpu = {"value": round(r, 3), "unit": "tok/s", "cores": threads, "kind": "oracle",
                "sample": f"{tokens} whole decode tokens (97 matrices each) in {dt:.1f} s, "
                          f"fp64 C oracle, OpenMP over output rows"}
+        r1, tokens1, dt1, _ = oracle_decode_tokens(host_weights, host_x, target_s=args.cpu_seconds, threads=1)
+        cpu1 = {"value": round(r1, 3), "unit": "tok/s", "cores": 1, "kind": "oracle",
+                "sample": f"{tokens1} whole decode tokens (97 matrices each) in {dt1:.1f} s, fp64 C oracle"}
+        if configs is not None:
+            for key, v in oracle_configs(threads).items():
+                configs.setdefault(key, {}).update(v)
 
     if world > 1:
         graph.reset()
@@ -390,7 +617,7 @@ def run_ours(args):
             "peak_kind": peak_kind,
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": None,
+            "traffic": measured_traffic(),
             "launches_per_step": dom["launches_per_step"],
             "bytes_per_launch": int(dom["bytes_per_launch"]),
             "avg_launch_us": round(dom["avg_launch_us"], 3),
@@ -412,6 +639,8 @@ def run_ours(args):
         "gpu_launches": len(specs) * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
+        "cpu_baseline_1thread": cpu1,
+        "configs": configs,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -425,6 +654,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (single GEMV, 7B small batch, MoE, Q8 x Q8)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

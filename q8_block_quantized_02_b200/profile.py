@@ -5,6 +5,7 @@
     python -m q8_block_quantized_02_b200.profile --op argmax --M 151936 --K 896 --N 1
     python -m q8_block_quantized_02_b200.profile --op moe --T 1
     python -m q8_block_quantized_02_b200.profile --op readpeak
+    python -m q8_block_quantized_02_b200.profile --op decode --reps 3
 
 Weights follow the synthetic Q8_0 recipe (q uniform in [-127, 127], d =
 |N(0,1)| * 0.02) and activations are N(0,1).  Enough packed copies of the
@@ -27,6 +28,11 @@ through them, so consecutive calls select different experts.  Bytes per
 call count each call's distinct selected experts plus the shared expert once
 (34 B per 32 weights).
 
+`--op decode` runs `--reps` decode steps of the Qwen2.5-0.5B matmul set (the
+benchmark's step: 24 x {qkv, wo, gate_up + SwiGLU, down} + lm_head, 97
+dependent launches on one stream), eagerly, after `--warmup` steps: the
+driver of ncu captures of the decode kernels in their chain.
+
 `--op readpeak` is a reference figure, not a libq8 product: the HBM read rate
 of a plain reduction (torch.sum over 4 GiB of fp32, so every byte is read
 once and nothing is written back), the read-only counterpart of the measured
@@ -46,7 +52,7 @@ if ROOT not in sys.path:
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--op", choices=["gemv", "argmax", "swiglu", "q8q8", "q4k", "q6k", "moe", "readpeak"],
+    ap.add_argument("--op", choices=["gemv", "argmax", "swiglu", "q8q8", "q4k", "q6k", "moe", "readpeak", "decode"],
                     default="gemv",
                     help="q8_gemv, q8_gemv_argmax (logits not written), q8_gate_up_swiglu (M = rows of "
                          "the stacked gate|up matrix) or q8_quantize_act + q8q8_gemv (only q8q8_gemv is "
@@ -70,6 +76,8 @@ def main(argv=None) -> int:
         return _moe(args)
     if args.op == "readpeak":
         return _readpeak(args)
+    if args.op == "decode":
+        return _decode(args)
 
     import numpy as np
     import torch
@@ -167,6 +175,47 @@ def _kquant(args, q8, q8gen, np, torch, dev) -> int:
     us = t0.elapsed_time(t1) * 1e3 / max(1, args.reps)
     print(json.dumps({"op": args.op, "M": M, "K": K, "N": N, "us_per_call": round(us, 3),
                       "weight_GBps": round(blocks.size / (us * 1e-6) / 1e9, 1), "copies": copies,
+                      "reps": args.reps, "device_error": word}), flush=True)
+    return 0 if st == 0 else 1
+
+
+def _decode(args) -> int:
+    import torch
+
+    import q8gen
+    import q8_block_quantized_02_b200 as q8
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    specs = q8gen.decode_matrices_05b()
+    packed, xs, ys = [], [], []
+    for s in specs:
+        g, x = q8gen.q8_matrix(s.seed, s.M, s.K, 1)
+        p = torch.empty(q8.q8_packed_bytes(s.M, s.K), dtype=torch.uint8, device=dev)
+        q8.q8_pack_weights(torch.from_numpy(g).to(dev), s.M, s.K, p)
+        packed.append(p)
+        xs.append(torch.from_numpy(x[0]).to(dev))
+        ys.append(torch.empty(s.M // 2 if s.swiglu else s.M, dtype=torch.float32, device=dev))
+
+    def step():
+        for i, s in enumerate(specs):
+            if s.swiglu:
+                q8.q8_gate_up_swiglu(packed[i], xs[i], ys[i], s.M // 2, s.K, 1)
+            else:
+                q8.q8_gemv(packed[i], xs[i], ys[i], s.M, s.K, 1)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.reps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    st, word = q8.q8_read_device_error()
+    us = t0.elapsed_time(t1) * 1e3 / max(1, args.reps)
+    print(json.dumps({"op": "decode", "launches_per_step": len(specs), "us_per_step_eager": round(us, 2),
                       "reps": args.reps, "device_error": word}), flush=True)
     return 0 if st == 0 else 1
 
