@@ -197,7 +197,8 @@ def _graph_time_us(torch, stream, calls, replays=5):
 
 def gpu_configs(q8, torch, dev, stream):
     """Device time per call of the single GEMV (1152x896, seed 0), the 7B-class
-    small-batch products (N = 1, 2, 4, 8, 16), the Qwen1.5-MoE block (T = 1, 8)
+    small-batch products (N = 1, 2, 4, 8, 16 through the default entry points,
+    N = 3, 4, 8, 16 through the split ones), the Qwen1.5-MoE block (T = 1, 8)
     and the Q8 x Q8 sweep (M = 4096, K in {896, 3584, 4864, 18944}, N in {1,
     16}).  Calls walk distinct packed copies of each matrix covering several
     times the L2 (the same bytes, so only the cache behaviour differs), or
@@ -237,16 +238,20 @@ def gpu_configs(q8, torch, dev, stream):
         ps = packed_copies(g, spec.M, spec.K, 2 * l2)
         rows = spec.M // 2 if spec.swiglu else spec.M
         res = {}
-        for N in (1, 2, 4, 8, 16):
+        # the default entry point (CUDA cores) at every N; the split entry
+        # point (tensor cores where faster) from N = 3
+        for N, split in [(n, False) for n in (1, 2, 4, 8, 16)] + [(n, True) for n in (3, 4, 8, 16)]:
             xd = torch.from_numpy(q8gen.activations(100 + N, N, spec.K)).to(dev)
             y = torch.empty((N, rows), dtype=torch.float32, device=dev)
             if spec.swiglu:
-                calls = [lambda p=p: q8.q8_gate_up_swiglu(p, xd, y, rows, spec.K, N, stream=stream) for p in ps]
+                fn = q8.q8_gate_up_swiglu_split if split else q8.q8_gate_up_swiglu
+                calls = [lambda p=p, fn=fn: fn(p, xd, y, rows, spec.K, N, stream=stream) for p in ps]
             else:
-                calls = [lambda p=p: q8.q8_gemv(p, xd, y, spec.M, spec.K, N, stream=stream) for p in ps]
+                fn = q8.q8_gemv_split if split else q8.q8_gemv
+                calls = [lambda p=p, fn=fn: fn(p, xd, y, spec.M, spec.K, N, stream=stream) for p in ps]
             us = _graph_time_us(torch, stream, calls * max(1, 4 // len(ps)))
-            res[f"N={N}"] = {"us_per_call": round(us, 2),
-                             "weight_GBps": round(algorithmic_bytes(spec.M, spec.K) / us / 1e3, 1)}
+            res[f"N={N}" + (",split" if split else "")] = {
+                "us_per_call": round(us, 2), "weight_GBps": round(algorithmic_bytes(spec.M, spec.K) / us / 1e3, 1)}
         key = f"7b_{spec.name}_{spec.M}x{spec.K}" + ("_swiglu" if spec.swiglu else "")
         out[key] = res
         del ps

@@ -120,23 +120,41 @@ q8_status q8_unpack_weights(const void *packed, int64_t M, int64_t K, void *gguf
 
 /* y[n][m] = sum_k d[m][k/32] * q[m][k] * x[n][k]   for n < N, m < M.
  * W: packed (q8_pack_weights) M x K.  x: [N][K] fp32.  y: [N][M] fp32, fully
- * overwritten.  fp32 arithmetic; each output is within 1e-5 * sum_k |w x| of
- * the exact value.  The Q8 N=1 decode product of "Lumen v0.3.0" (Phase 7.G)
- * and the "skuznetsov/cogni-ml" cuda_q8_gemv_probe ("Build Qwen CLIs"),
- * extended to N <= 16 columns.  N > 16 -> Q8_ERR_UNSUPPORTED.
- * N <= 4: fp32 dequantise-and-FMA on the CUDA cores.  5 <= N <= 16: the
- * tensor cores (tcgen05.mma kind::i8, one MMA per Q8_0 block) take the packed
- * int8 q against an exact three-term int8 split of each 32-block of x,
- * x = s (q0 + q1/254 + q2/254^2) with a power-of-two s per block (residual
- * below 2.5e-7 of the block's max |x|), and an fp32 epilogue applies d and s
- * per block.  There the split adds at most 2.5e-7 * sum_b amax_b * sum_{k in b}
- * |w_k| (amax_b: block b's max |x|) to the fp32 error: within the 1e-5 bar
- * for ordinary activations (all tests, including blocks of tiny values with
- * one large one), but not for every crafted input -- e.g. a block whose only
- * large value meets a zero weight.  Blocks whose max |x| is below 2^-121 lose
- * relative accuracy there; non-finite x is undefined. */
+ * overwritten.  fp32 arithmetic on the CUDA cores, and its only error is
+ * rounding: each weight d * q is exact in fp32, and each output is a sum of
+ * fp32 products in a fixed order (16-term packed dots, a chain per lane over
+ * its columns, then shuffle and cross-warp sums), so |y - y_exact| <=
+ * D * 2^-24 * sum_k |w x| for every input, D the longest chain of roundings:
+ * D <= K/512 + 30 for N <= 4 (1e-5 * sum|w x| up to K = 70000) and
+ * D <= K/64 + 30 for 5 <= N <= 16 (up to K = 8800; at K = 18944 the worst
+ * case is 1.9e-5 * sum|w x|).  Typical errors are far smaller (the tests
+ * measure below 1e-6 * sum|w x| at every shape).  The Q8 N=1 decode product
+ * of "Lumen v0.3.0" (Phase 7.G) and the "skuznetsov/cogni-ml"
+ * cuda_q8_gemv_probe ("Build Qwen CLIs"), extended to N <= 16 columns.
+ * N > 16 -> Q8_ERR_UNSUPPORTED.  Bit-identical results from run to run.
+ * See q8_gemv_split for the tensor-core variant. */
 q8_status q8_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
                   q8_stream_t stream);
+
+/* q8_gemv with the tensor cores allowed: where it is faster (N >= 5, or
+ * N >= 3 for matrices with at least 148 tiles of 128 rows), tcgen05.mma
+ * kind::i8 takes the packed int8 q against an exact-scale three-term int8
+ * split of each 32-block of x, x = s (q0 + q1/254 + q2/254^2) with a
+ * power-of-two s per block, one MMA per Q8_0 block and an fp32 epilogue that
+ * applies d and s; elsewhere it is q8_gemv.  The split's residual is below
+ * 2.5e-7 of the block's max |x|, so it adds at most
+ *   2.5e-7 * sum_b amax_b * sum_{k in b} |w_k|     (amax_b: block b's max |x|)
+ * to the fp32 error: far inside the 1e-5 * sum_k |w x| bar for activations
+ * whose blocks carry no value much larger than the rest at a near-zero
+ * weight, but that bar is not guaranteed for every input (a block whose only
+ * large value meets a zero weight breaks it), which is why this is a
+ * separate entry point.  x -> 2x still doubles y bit for bit, and unit-scale
+ * one-hot inputs come out exactly.  Blocks whose max |x| is below 2^-121
+ * lose relative accuracy; non-finite x is undefined.  Shapes and limits as
+ * q8_gemv.  Measured on the 7B-class shapes: 37888x3584 SwiGLU at N = 4 /
+ * 8 / 16 in 49 / 59 / 83 us (CUDA cores: 77 / 92 / 197 us). */
+q8_status q8_gemv_split(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                        q8_stream_t stream);
 
 /* y[n][m] = (W x)[n][m] + residual[n][m]: the q8_gemv product with the
  * residual-stream add of the projections that feed it (attention output and
@@ -215,10 +233,16 @@ q8_status q8_q6k_gemv(const void *W, const float *x, float *y, int64_t M, int64_
  * projections of the "skuznetsov/cogni-ml" FFN probe, "Build Qwen CLIs"; the
  * SwiGLU MLP of the "augur" README, "Features").  I must be a multiple of 8.
  * x: [N][K] fp32.  h: [N][I] fp32, fully overwritten.  One launch; g and u
- * never leave the chip.  5 <= N <= 16 runs on the tensor cores as q8_gemv
- * does (a tile holds 64 gate rows and their 64 up rows). */
+ * never leave the chip.  g and u each within q8_gemv's bound; h within the
+ * bound that carries through silu and the product. */
 q8_status q8_gate_up_swiglu(const void *W, const float *x, float *h, int64_t I, int64_t K,
                             int64_t N, q8_stream_t stream);
+
+/* q8_gate_up_swiglu with the tensor cores allowed, as q8_gemv_split (a tile
+ * holds 64 gate rows and their 64 up rows; g and u carry q8_gemv_split's
+ * bound). */
+q8_status q8_gate_up_swiglu_split(const void *W, const float *x, float *h, int64_t I, int64_t K,
+                                  int64_t N, q8_stream_t stream);
 
 /* ---------------------------------------------------------------------- */
 /* S5  MoE router                                                          */

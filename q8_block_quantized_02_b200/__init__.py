@@ -25,7 +25,7 @@ __all__ = [
     "q8_moe_gemv",
     "q8_moe_gemv_noalloc",
     "q8_quantize_act", "q8_rmsnorm_quantize_act", "q8q8_gemv", "q8q8_block_dots",
-    "q8_test_wait_timeout",
+    "q8_test_wait_timeout", "q8_gemv_split", "q8_gate_up_swiglu_split",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -64,6 +64,8 @@ _SIGS = {
     "q8_rmsnorm_quantize_act": (_INT, [_P, _P, ctypes.c_float, _P, _P, _P, _I64, _I64, _P]),
     "q8q8_block_dots": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "q8_test_wait_timeout": (_INT, [ctypes.c_uint32, _P, _P]),
+    "q8_gemv_split": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
+    "q8_gate_up_swiglu_split": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
 }
 
 
@@ -249,3 +251,11 @@ def q8q8_block_dots(W, xq, dots, M, K, N, stream=None):
 
 def q8_test_wait_timeout(limit_us, out, stream=None):
     _call("q8_test_wait_timeout", int(limit_us), _ptr(out), _stream(stream))
+
+
+def q8_gemv_split(W, x, y, M, K, N, stream=None):
+    _call("q8_gemv_split", _ptr(W), _ptr(x), _ptr(y), M, K, N, _stream(stream))
+
+
+def q8_gate_up_swiglu_split(W, x, h, I, K, N, stream=None):
+    _call("q8_gate_up_swiglu_split", _ptr(W), _ptr(x), _ptr(h), I, K, N, _stream(stream))

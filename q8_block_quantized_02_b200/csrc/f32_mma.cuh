@@ -56,7 +56,8 @@
 // boxes of the first stages before griddepcontrol.wait), 1 owns tensor memory
 // and issues the MMAs, 2..9 split (warp 2 + i takes activation rows i and
 // i + 8), 10..25 are the epilogue: warp w reads TMEM lanes 32 * (w % 4) .. and
-// TOK activation rows from TOK * ((w - 10) / 4) (TOK = 2 for N <= 8, else 4),
+// TOK activation rows from TOK * ((w - 10) / 4) (TOK = 1 for N <= 4, 2 for
+// N <= 8, else 4),
 // so the epilogue's work spreads over 16 warps at any N, and no epilogue warp
 // waits for a split.  With fewer 128-row tiles than
 // SMs, K is split over a cluster of up to 8 CTAs and the partial sums meet in
@@ -132,6 +133,9 @@ __device__ __forceinline__ void tmem_ld4_async(uint32_t taddr, uint32_t *v) {
                  : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
                  : "r"(taddr)
                  : "memory");
+}
+__device__ __forceinline__ void tmem_ld1_async(uint32_t taddr, uint32_t *v) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v[0]) : "r"(taddr) : "memory");
 }
 __device__ __forceinline__ void tmem_ld2_async(uint32_t taddr, uint32_t *v) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];"
@@ -266,12 +270,12 @@ __device__ __forceinline__ void fm_epilogue_blocks(float (&acc)[TOK], const uint
     }
 }
 
-// TOK: activation rows per epilogue warp (2 for N <= 8, else 4).
+// TOK: activation rows per epilogue warp (1 for N <= 4, 2 for N <= 8, else 4).
 template <bool SWIGLU, int TOK>
 __global__ void __launch_bounds__(kFmThreads, 1)
     f32_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap td,
                    const float *__restrict__ x, const FmArgs a) {
-    constexpr int LB = 8 / TOK;  // blocks per TMEM load batch (24 registers)
+    constexpr int LB = TOK == 1 ? 4 : 8 / TOK;  // blocks per TMEM load batch (at most 24 registers)
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = a.split;
@@ -485,8 +489,10 @@ __global__ void __launch_bounds__(kFmThreads, 1)
                                     const uint32_t ta = taddr + (jb + jj) * kFmBlockCols + k * kFmN;
                                     if (TOK == 4)
                                         tmem_ld4_async(ta, v[jj][k]);
-                                    else
+                                    else if (TOK == 2)
                                         tmem_ld2_async(ta, v[jj][k]);
+                                    else
+                                        tmem_ld1_async(ta, v[jj][k]);
                                 }
                             uint32_t *vf = &v[0][0][0];
                             tmem_wait_ld8(vf);

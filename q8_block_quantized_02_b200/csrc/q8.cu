@@ -328,22 +328,37 @@ static q8_status run_resident(const TilePlan &plan, const void *W, const float *
 static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_out, int64_t K,
                         int64_t N, bool swiglu, cudaStream_t stream, const float *res);
 
-#ifndef Q8_FM_MIN_N
-#define Q8_FM_MIN_N 5
-#endif
-constexpr int64_t kFmMinN = Q8_FM_MIN_N;  // smallest N of fp32 activations sent to the tensor cores
+constexpr int64_t kFmMinN = 5;       // smallest N the split entry points always send to the tensor cores
+constexpr int64_t kFmMinNLarge = 3;  // ... and for matrices with a 128-row tile per SM or more
+
+// The split entry points (q8_gemv_split, q8_gate_up_swiglu_split) send fp32
+// activations to the tensor-core kernel from N = 5, and from N = 3 when the
+// matrix has at least one output tile per SM (no K split): measured on the
+// 7B-class shapes, 37888x3584 SwiGLU at N = 3 / 4 takes 46 / 49 us there
+// against 69 / 77 us on the CUDA cores, 152064x3584 186 / 197 us against
+// 259 / 291 us; the 3584x18944 down projection (28 tiles, K split over
+// clusters) stays faster on the CUDA cores below N = 5 (42 / 48 us against
+// 54 / 58 us).  The default entry points keep every N on the CUDA cores, whose
+// error bound is relative to sum |w x| for every input.
+static bool fm_serves(int64_t rows_out, int64_t N, bool swiglu, int sms) {
+    if (N >= kFmMinN) return true;
+    const int64_t tiles = ceil_div(rows_out, swiglu ? 64 : 128);
+    return N >= kFmMinNLarge && tiles >= sms;
+}
 
 // `best` (fp32 GEMV, N <= 4 only): also leave the arg-max key of every
 // column there (q8_gemv_argmax); the column-owner kernel serves it.
 // `res` (fp32 GEMV): added to every output (q8_gemv_residual).
+// `split` (fp32 modes): the tensor-core kernel with the three-term int8 split
+// of x may serve the call where it is faster (fm_serves).
 static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, float *y,
                           int64_t rows_out, int64_t K, int64_t N, int mode, cudaStream_t stream,
-                          unsigned long long *best = nullptr, const float *res = nullptr) {
+                          unsigned long long *best = nullptr, const float *res = nullptr, bool split = false) {
     const bool swiglu = mode == kModeSwiGLU;
-    if (mode != kModeQ8Q8 && N >= kFmMinN && !best)
-        return run_fm(W, static_cast<const float *>(x), y, rows_out, K, N, swiglu, stream, res);
     const DeviceInfo *dev = nullptr;
     Q8_CHECK(device_info(&dev));
+    if (split && mode != kModeQ8Q8 && !best && fm_serves(rows_out, N, swiglu, dev->sms))
+        return run_fm(W, static_cast<const float *>(x), y, rows_out, K, N, swiglu, stream, res);
     const int64_t B = K / 32, C = K / 16;
     const int64_t units = ceil_div(rows_out, kGroupRows);
     const int64_t total_groups = swiglu ? 2 * units : units;
@@ -471,8 +486,10 @@ static q8_status run_mma(const void *W, const int8_t *xq, const uint16_t *xd, fl
 // fp32 activations on the tensor cores (S3 / S4, 5..16 activation columns)
 // ---------------------------------------------------------------------------
 static cudaError_t setup_fm_kernels(int max_smem) {
-    const void *ks[4] = {reinterpret_cast<const void *>(&f32_mma_kernel<false, 2>),
+    const void *ks[6] = {reinterpret_cast<const void *>(&f32_mma_kernel<false, 1>),
+                         reinterpret_cast<const void *>(&f32_mma_kernel<false, 2>),
                          reinterpret_cast<const void *>(&f32_mma_kernel<false, 4>),
+                         reinterpret_cast<const void *>(&f32_mma_kernel<true, 1>),
                          reinterpret_cast<const void *>(&f32_mma_kernel<true, 2>),
                          reinterpret_cast<const void *>(&f32_mma_kernel<true, 4>)};
     for (const void *k : ks) {
@@ -544,10 +561,10 @@ static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_ou
     Q8_CHECK(make_map_3d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT16, dbase, 8, B, groups, 16, gstride, 8,
                          kFmSB, 8, true));
     // the activations are read by the kernel's splitter warps with plain loads;
-    // each epilogue warp takes 2 activation rows up to N = 8, else 4
+    // each epilogue warp takes 1 activation row up to N = 4, 2 up to N = 8, else 4
     using FmKernel = void (*)(CUtensorMap, CUtensorMap, const float *, FmArgs);
-    const FmKernel k = swiglu ? (N <= 8 ? &f32_mma_kernel<true, 2> : &f32_mma_kernel<true, 4>)
-                              : (N <= 8 ? &f32_mma_kernel<false, 2> : &f32_mma_kernel<false, 4>);
+    const FmKernel k = swiglu ? (N <= 4 ? &f32_mma_kernel<true, 1> : N <= 8 ? &f32_mma_kernel<true, 2> : &f32_mma_kernel<true, 4>)
+                              : (N <= 4 ? &f32_mma_kernel<false, 1> : N <= 8 ? &f32_mma_kernel<false, 2> : &f32_mma_kernel<false, 4>);
     return launch_pdl_cluster(k, dim3(p.grid), dim3(kFmThreads), p.smem, stream,
                               swiglu ? "q8_gate_up_swiglu (tensor cores) launch" : "q8_gemv (tensor cores) launch",
                               (unsigned)p.a.split, tq, td, x, p.a);
@@ -870,6 +887,16 @@ q8_status q8_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K,
     return run_tile(W, x, nullptr, y, M, K, N, kModeF32, (cudaStream_t)stream);
 }
 
+q8_status q8_gemv_split(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                        q8_stream_t stream) {
+    if (M <= 0 || K <= 0 || N <= 0 || K % 32) return Q8_ERR_SHAPE;
+    if (N > 16 || M > (int64_t)1 << 30 || K > (int64_t)1 << 24) return Q8_ERR_UNSUPPORTED;
+    Q8_CHECK(check_device_ptr(W));
+    Q8_CHECK(check_device_ptr(x));
+    Q8_CHECK(check_device_ptr(y));
+    return run_tile(W, x, nullptr, y, M, K, N, kModeF32, (cudaStream_t)stream, nullptr, nullptr, true);
+}
+
 q8_status q8_q4k_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
                       q8_stream_t stream) {
     return run_kquant<4>(W, x, y, M, K, N, (cudaStream_t)stream, "q8_q4k_gemv launch");
@@ -918,6 +945,16 @@ q8_status q8_gate_up_swiglu(const void *W, const float *x, float *h, int64_t I, 
     Q8_CHECK(check_device_ptr(x));
     Q8_CHECK(check_device_ptr(h));
     return run_tile(W, x, nullptr, h, I, K, N, kModeSwiGLU, (cudaStream_t)stream);
+}
+
+q8_status q8_gate_up_swiglu_split(const void *W, const float *x, float *h, int64_t I, int64_t K,
+                                  int64_t N, q8_stream_t stream) {
+    if (I <= 0 || K <= 0 || N <= 0 || K % 32 || I % 8) return Q8_ERR_SHAPE;
+    if (N > 16 || I > (int64_t)1 << 29 || K > (int64_t)1 << 24) return Q8_ERR_UNSUPPORTED;
+    Q8_CHECK(check_device_ptr(W));
+    Q8_CHECK(check_device_ptr(x));
+    Q8_CHECK(check_device_ptr(h));
+    return run_tile(W, x, nullptr, h, I, K, N, kModeSwiGLU, (cudaStream_t)stream, nullptr, nullptr, true);
 }
 
 q8_status q8_quantize_act(const float *x, int8_t *xq, uint16_t *xd, int64_t N, int64_t K,

@@ -37,23 +37,25 @@ def pack(gguf: np.ndarray, M: int, K: int):
     return packed
 
 
-def gemv(packed, x: np.ndarray, M: int, K: int):
+def gemv(packed, x: np.ndarray, M: int, K: int, split: bool = False):
+    """q8_gemv (or, with split, q8_gemv_split) on x; returns y [N][M]."""
     import q8_block_quantized_02_b200 as q8
     t = torch()
     xd = dev(x.astype(np.float32))
     N = x.shape[0]
     y = t.full((N, M), float("nan"), dtype=t.float32, device="cuda")
-    q8.q8_gemv(packed, xd, y, M, K, N)
+    (q8.q8_gemv_split if split else q8.q8_gemv)(packed, xd, y, M, K, N)
     return y.cpu().numpy()
 
 
-def gate_up(packed, x: np.ndarray, I: int, K: int):
+def gate_up(packed, x: np.ndarray, I: int, K: int, split: bool = False):
+    """q8_gate_up_swiglu (or its split variant) on x; returns h [N][I]."""
     import q8_block_quantized_02_b200 as q8
     t = torch()
     xd = dev(x.astype(np.float32))
     N = x.shape[0]
     h = t.full((N, I), float("nan"), dtype=t.float32, device="cuda")
-    q8.q8_gate_up_swiglu(packed, xd, h, I, K, N)
+    (q8.q8_gate_up_swiglu_split if split else q8.q8_gate_up_swiglu)(packed, xd, h, I, K, N)
     return h.cpu().numpy()
 
 

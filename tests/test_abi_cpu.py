@@ -166,6 +166,14 @@ def test_host_validation_runs_before_any_device_work(lib):
     assert am(n, n, n, 8, 33, 1, n, n) == 2
     assert am(n, n, n, 8, 32, 5, n, n) == 5         # N > 4
     assert am(n, n, n, 8, 32, 4, n, n) == 1
+    gs = fn("q8_gemv_split", P, P, P, I64, I64, I64, P)
+    assert gs(n, n, n, 8, 48, 1, n) == 2
+    assert gs(n, n, n, 8, 32, 17, n) == 5
+    assert gs(n, n, n, 8, 32, 4, n) == 1
+    ss = fn("q8_gate_up_swiglu_split", P, P, P, I64, I64, I64, P)
+    assert ss(n, n, n, 12, 32, 1, n) == 2
+    assert ss(n, n, n, 16, 32, 17, n) == 5
+    assert ss(n, n, n, 16, 32, 8, n) == 1
     sw = fn("q8_gate_up_swiglu", P, P, P, I64, I64, I64, P)
     assert sw(n, n, n, 12, 32, 1, n) == 2           # I % 8
     assert sw(n, n, n, 16, 32, 17, n) == 5

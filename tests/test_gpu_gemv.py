@@ -71,10 +71,8 @@ SHAPES = [
 ]
 
 
-# every shape at N <= 4; at N = 8 and 16 (the tensor-core path, which has its
-# own file of shapes) only the shapes up to 1152 x 896 x 8 products
-GEMV_CASES = [(M, K, N) for N in (1, 2, 3, 4, 8, 16) for (M, K) in SHAPES
-              if N <= 4 or M * K * N <= 1152 * 896 * 8]
+# every shape at every N (N >= 5: the group-owner kernel on the CUDA cores)
+GEMV_CASES = [(M, K, N) for N in (1, 2, 3, 4, 5, 8, 16) for (M, K) in SHAPES]
 
 
 @pytest.mark.parametrize("M,K,N", GEMV_CASES)
@@ -154,11 +152,11 @@ def test_gemv_full_size_sampled(M, K):
 
 
 @pytest.mark.parametrize("M,K", [(152064, 3584), (3584, 18944)])
-@pytest.mark.parametrize("N", [2, 4])
+@pytest.mark.parametrize("N", [2, 4, 8, 16])
 def test_gemv_full_size_sampled_small_batch(M, K, N):
-    """The 7B-class lm_head and down at N = 2 and 4 (the small-batch sweep's
-    CUDA-core columns), full size, at the launch shape the planner picks for
-    them; sampled rows against the oracle."""
+    """The 7B-class lm_head and down at N = 2, 4, 8 and 16 (the small-batch
+    sweep), full size, at the launch shape the planner picks for them on the
+    CUDA cores; sampled rows against the oracle."""
     g, x = matrix(3030 + M + N, M, K, N)
     y = gemv(pack(g, M, K), x, M, K)
     rng = np.random.default_rng(N)
@@ -173,9 +171,7 @@ def test_gemv_full_size_sampled_small_batch(M, K, N):
 # --------------------------------------------------------------------------
 
 SWIGLU_SHAPES = [(4864, 896), (8, 32), (1408, 2048), (104, 4864), (200, 896)]
-# every shape at N <= 2; at N = 5 and 16 (the tensor-core path) the smaller ones
-SWIGLU_CASES = [(I, K, N) for N in (1, 2, 5, 16) for (I, K) in SWIGLU_SHAPES
-                if N <= 2 or I * K * N <= 4864 * 896 * 2]
+SWIGLU_CASES = [(I, K, N) for N in (1, 2, 5, 8, 16) for (I, K) in SWIGLU_SHAPES]
 
 
 @pytest.mark.parametrize("I,K,N", SWIGLU_CASES)
@@ -186,9 +182,9 @@ def test_gate_up_swiglu_matches_oracle(I, K, N):
     assert_within(h, ref["h"], swiglu_bound(ref), f"swiglu I={I} K={K} N={N}")
 
 
-@pytest.mark.parametrize("N", [1, 2, 4])
+@pytest.mark.parametrize("N", [1, 2, 4, 8, 16])
 def test_gate_up_full_size_sampled(N):
-    """7B-class gate_up (37888 x 3584) at N = 1, 2 and 4, sampled rows."""
+    """7B-class gate_up (37888 x 3584) at N = 1, 2, 4, 8 and 16, sampled rows."""
     I, K = 18944, 3584
     g, x = matrix(4242 + (N - 1) * 7, 2 * I, K, N)
     h = gate_up(pack(g, 2 * I, K), x, I, K)
