@@ -217,11 +217,13 @@ __device__ __forceinline__ void tile_produce(uint8_t *smem, uint32_t full0, uint
     // scales (two TMA instructions: each costs tens of ns to issue); the
     // partial last tile of a CTA's range is fetched unit by unit so that
     // nothing outside the range is read.
-    auto issue_weights = [&](int it) {
-        const int slot = it % a.stages;
-        const int ut = u0 + (it / a.ksteps) * a.TG;
+    // The ring position (slot, phase) and the tile position (tile, k step) of
+    // iteration `it` are carried along, not divided out of `it` (an integer
+    // division by a runtime value costs tens of instructions).
+    auto issue_weights = [&](int slot, int tile, int ks) {
+        const int ut = u0 + tile * a.TG;
         const int tga = min(a.TG, u1 - ut);
-        const int c0 = (it % a.ksteps) * a.CS;
+        const int c0 = ks * a.CS;
         const uint32_t st = smem_u32(smem + (size_t)slot * a.stage_bytes);
         const uint32_t full = full0 + 8 * slot;
         mbar_arrive_expect_tx(full, HALVES * tga * (a.q_box + a.d_box) + a.x_box);
@@ -240,21 +242,31 @@ __device__ __forceinline__ void tile_produce(uint8_t *smem, uint32_t full0, uint
             }
         }
     };
-    auto issue_x = [&](int it) {
-        const int slot = it % a.stages;
+    auto issue_x = [&](int slot, int ks) {
         const uint32_t st = smem_u32(smem + (size_t)slot * a.stage_bytes);
-        tma_load_3d(st + a.x_off, tx, full0 + 8 * slot, 0, (it % a.ksteps) * a.CS, 0, px);
+        tma_load_3d(st + a.x_off, tx, full0 + 8 * slot, 0, ks * a.CS, 0, px);
     };
     const int pro = total < a.stages ? total : a.stages;
-    int it = 0;
-    for (; it < pro; ++it) issue_weights(it);  // weights never depend on the previous grid
-    pdl_wait_and_trigger();                    // activations may
-    for (int k = 0; k < pro; ++k) issue_x(k);
+    int it = 0, tile = 0, ks = 0;
+    for (; it < pro; ++it) {  // weights never depend on the previous grid
+        issue_weights(it, tile, ks);
+        if (++ks == a.ksteps) { ks = 0; ++tile; }
+    }
+    pdl_wait_and_trigger();  // activations may
+    {
+        int kx = 0;
+        for (int k = 0; k < pro; ++k) {
+            issue_x(k, kx);
+            if (++kx == a.ksteps) kx = 0;
+        }
+    }
+    int slot = pro % a.stages, phase = pro / a.stages;  // ring position of iteration `pro`
     for (; it < total; ++it) {
-        const int slot = it % a.stages;
-        if (!mbar_wait(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag)) break;
-        issue_weights(it);
-        issue_x(it);
+        if (!mbar_wait(empty0 + 8 * slot, (phase & 1) ^ 1, abort_flag)) break;
+        issue_weights(slot, tile, ks);
+        issue_x(slot, ks);
+        if (++ks == a.ksteps) { ks = 0; ++tile; }
+        if (++slot == a.stages) { slot = 0; ++phase; }
     }
     *issued = it;
 }
@@ -459,7 +471,7 @@ __global__ void __launch_bounds__(ColsCfg<NMAX, MODE, CW_>::THREADS, 1)
         // ------------------------------ consumers -----------------------------
         const int cw = warp, cg = cw / WPG, lw = cw % WPG, r = lane & 7, j = lane >> 3;
         pdl_wait_and_trigger();  // Q8Q8: activation scales are read straight from memory
-        int it = 0;
+        int it = 0, slot = 0, phase = 0;  // ring position of iteration `it`, carried along
         for (int tl = 0; tl < n_tiles; ++tl) {
             const int ut = u0 + tl * a.TG;
             const int tga = min(a.TG, u1 - ut);
@@ -470,9 +482,9 @@ __global__ void __launch_bounds__(ColsCfg<NMAX, MODE, CW_>::THREADS, 1)
                 for (int h = 0; h < H; ++h)
 #pragma unroll
                     for (int n = 0; n < NMAX; ++n) acc[g][h][n] = 0.f;
-            for (int ks = 0; ks < a.ksteps; ++ks, ++it) {
+            for (int ks = 0; ks < a.ksteps;
+                 ++ks, ++it, slot = slot + 1 == a.stages ? 0 : slot + 1, phase ^= slot == 0 ? 1 : 0) {
                 if (it % Cfg::GROUPS != cg) continue;
-                const int slot = it % a.stages;
                 // With two groups a slot can pass from one group to the other
                 // (odd ring): wait for the release of the slot's previous
                 // stage, as the producer does, before waiting for this fill.
@@ -480,8 +492,8 @@ __global__ void __launch_bounds__(ColsCfg<NMAX, MODE, CW_>::THREADS, 1)
                 // phase of `full` has the parity this wait asks for.
                 bool ready = true;
                 if (Cfg::GROUPS > 1 && it >= a.stages)
-                    ready = mbar_wait(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag);
-                if (ready && mbar_wait(full0 + 8 * slot, (it / a.stages) & 1, abort_flag)) {
+                    ready = mbar_wait(empty0 + 8 * slot, phase ^ 1, abort_flag);
+                if (ready && mbar_wait(full0 + 8 * slot, phase, abort_flag)) {
                     const uint8_t *st = smem + (size_t)slot * a.stage_bytes;
                     const int cols = min(a.CS, a.C - ks * a.CS);
                     const int nq = (cols + 3) >> 2;
@@ -538,7 +550,7 @@ __device__ __forceinline__ void consume_groups(uint8_t *smem, uint32_t full0, ui
     constexpr int SETS = tile_acc_sets<MODE>();
     const int cw = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane & 7, j = lane >> 3;
     pdl_wait_and_trigger();  // outputs may still be read by the previous grid
-    int it = 0;
+    int it = 0, slot = 0, phase = 0;  // ring position of iteration `it`, carried along
     for (int tl = 0; tl < n_tiles; ++tl) {
         const int ut = u0 + tl * a.TG;
         const int tga = min(a.TG, u1 - ut);
@@ -552,9 +564,9 @@ __device__ __forceinline__ void consume_groups(uint8_t *smem, uint32_t full0, ui
         for (int h = 0; h < SETS; ++h)
 #pragma unroll
             for (int n = 0; n < NMAX; ++n) acc[h][n] = 0.f;
-        for (int ks = 0; ks < a.ksteps; ++ks, ++it) {
-            const int slot = it % a.stages;
-            if (mbar_wait(full0 + 8 * slot, (it / a.stages) & 1, abort_flag)) {
+        for (int ks = 0; ks < a.ksteps;
+             ++ks, ++it, slot = slot + 1 == a.stages ? 0 : slot + 1, phase ^= slot == 0 ? 1 : 0) {
+            if (mbar_wait(full0 + 8 * slot, phase, abort_flag)) {
                 const uint8_t *st = smem + (size_t)slot * a.stage_bytes;
                 const int cols = min(a.CS, a.C - ks * a.CS);
                 const int nq = (cols + 3) >> 2;
