@@ -354,10 +354,11 @@ __global__ void __launch_bounds__(kFmThreads, 1)
         // --------------------------- producer (weights) ---------------------------
         if (lane == 0 && total > 0) {
             const uint64_t pw = policy_evict_first();
-            auto issue_w = [&](int it) {
-                const int slot = it % a.stages;
-                const int tile = t0 + it / ksteps;
-                const int b0 = b_lo + (it % ksteps) * kFmSB;
+            // ring slot/phase and (tile, k step) are carried along: no
+            // division by a runtime value per stage
+            auto issue_w = [&](int slot, int tile_i, int ks) {
+                const int tile = t0 + tile_i;
+                const int b0 = b_lo + ks * kFmSB;
                 const uint32_t st = smem_u32(smem + (size_t)slot * kFmStageBytes);
                 const uint32_t full = full0 + 8 * slot;
                 const int ga = SWIGLU ? 8 * tile : 16 * tile;
@@ -369,13 +370,18 @@ __global__ void __launch_bounds__(kFmThreads, 1)
                 tma_load_3d(st + kFmDOff + kFmDBox, &td, full, 0, b0, gb, pw);
             };
             const int pro = total < a.stages ? total : a.stages;
-            int it = 0;
-            for (; it < pro; ++it) issue_w(it);  // weights never depend on the previous grid
+            int it = 0, tile = 0, ks = 0;
+            for (; it < pro; ++it) {  // weights never depend on the previous grid
+                issue_w(it, tile, ks);
+                if (++ks == ksteps) { ks = 0; ++tile; }
+            }
             pdl_wait_and_trigger();
+            int slot = pro % a.stages, phase = pro / a.stages;  // ring position of iteration `pro`
             for (; it < total; ++it) {
-                const int slot = it % a.stages;
-                if (!mbar_wait(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag)) break;
-                issue_w(it);
+                if (!mbar_wait(empty0 + 8 * slot, (phase & 1) ^ 1, abort_flag)) break;
+                issue_w(slot, tile, ks);
+                if (++ks == ksteps) { ks = 0; ++tile; }
+                if (++slot == a.stages) { slot = 0; ++phase; }
             }
             *issued = it;
         } else {
@@ -386,12 +392,15 @@ __global__ void __launch_bounds__(kFmThreads, 1)
         pdl_wait_and_trigger();
         if (lane == 0) {
             bool ok = true;
-            for (int it = 0; it < total && ok; ++it) {
-                const int slot = it % a.stages, ab = it % kFmNB;
-                if (!mbar_wait(full0 + 8 * slot, (it / a.stages) & 1, abort_flag)) break;
+            int slot = 0, phase = 0, ks = 0;  // ring position and k step of iteration `it`
+            for (int it = 0; it < total && ok;
+                 ++it, ks = ks + 1 == ksteps ? 0 : ks + 1, slot = slot + 1 == a.stages ? 0 : slot + 1,
+                     phase ^= slot == 0 ? 1 : 0) {
+                const int ab = it % kFmNB;
+                if (!mbar_wait(full0 + 8 * slot, phase, abort_flag)) break;
                 if (!mbar_wait(bready0 + 8 * ab, (it / kFmNB) & 1, abort_flag)) break;
                 tc_fence_after();
-                const int nb = min(kFmSB, nblk - (it % ksteps) * kFmSB);
+                const int nb = min(kFmSB, nblk - ks * kFmSB);
                 const uint32_t st = smem_u32(smem + (size_t)slot * kFmStageBytes);
                 const uint32_t xb = smem_u32(act + ab * kFmActBytes);
                 for (int h = 0; h < kFmHalves; ++h) {
@@ -427,19 +436,19 @@ __global__ void __launch_bounds__(kFmThreads, 1)
         const int K = 32 * a.B;
         pdl_wait_and_trigger();   // the activations belong to the previous grid until now
         uint4 xr[2][2];
-        auto load = [&](int it) {
-            const int ks = it % ksteps, b0 = b_lo + ks * kFmSB, nb = min(kFmSB, nblk - ks * kFmSB);
+        auto load = [&](int ks) {
+            const int b0 = b_lo + ks * kFmSB, nb = min(kFmSB, nblk - ks * kFmSB);
             fm_load_x(x, K, sw, a.N, b0, nb, lane, xr[0]);
             fm_load_x(x, K, sw + 8, a.N, b0, nb, lane, xr[1]);
         };
         if (total > 0) load(0);
-        for (int it = 0; it < total; ++it) {
+        for (int it = 0, ks = 0; it < total; ++it, ks = ks + 1 == ksteps ? 0 : ks + 1) {
             const int ab = it % kFmNB;
             // the buffer's previous stage (it - kFmNB) has been read by its MMAs and epilogue
             const bool ok =
                 it < kFmNB || mbar_wait_warp(bfree0 + 8 * ab, ((it / kFmNB) - 1) & 1, abort_flag);
             if (ok) {
-                const int nb = min(kFmSB, nblk - (it % ksteps) * kFmSB);
+                const int nb = min(kFmSB, nblk - ks * kFmSB);
                 uint8_t *abuf = act + ab * kFmActBytes;
                 if (sw < a.N) fm_split_row(abuf, xr[0], sw, lane, nb);
                 if (sw + 8 < a.N) fm_split_row(abuf, xr[1], sw + 8, lane, nb);
@@ -447,7 +456,7 @@ __global__ void __launch_bounds__(kFmThreads, 1)
             fence_proxy_async_smem();  // the MMA reads the pieces through the async proxy
             __syncwarp();
             if (lane == 0) mbar_arrive(bready0 + 8 * ab);
-            if (it + 1 < total) load(it + 1);  // lands while this stage's pieces are consumed
+            if (it + 1 < total) load(ks + 1 == ksteps ? 0 : ks + 1);  // lands while this stage's pieces are consumed
         }
     } else {
         // ------------------------------ epilogue ------------------------------
@@ -460,18 +469,19 @@ __global__ void __launch_bounds__(kFmThreads, 1)
         const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + n0;
         pdl_wait_and_trigger();  // the outputs belong to the previous grid until now
         float acc[TOK];
-        int it = 0;
+        int it = 0, slot = 0, phase = 0;  // ring position of iteration `it`, carried along
         for (int tl = 0; tl < n_tiles; ++tl) {
 #pragma unroll
             for (int t = 0; t < TOK; ++t) acc[t] = 0.f;
-            for (int ks = 0; ks < ksteps; ++ks, ++it) {
-                const int slot = it % a.stages, ab = it % kFmNB;
+            for (int ks = 0; ks < ksteps;
+                 ++ks, ++it, slot = slot + 1 == a.stages ? 0 : slot + 1, phase ^= slot == 0 ? 1 : 0) {
+                const int ab = it % kFmNB;
                 const uint8_t *st = smem + (size_t)slot * kFmStageBytes;
                 const uint8_t *abuf = act + ab * kFmActBytes;
                 // the stage's table entries are written, and its weights (their
                 // scales) have landed
                 bool ok = mbar_wait_warp(bready0 + 8 * ab, (it / kFmNB) & 1, abort_flag);
-                ok = ok && mbar_wait_warp(full0 + 8 * slot, (it / a.stages) & 1, abort_flag);
+                ok = ok && mbar_wait_warp(full0 + 8 * slot, phase, abort_flag);
                 const int nb = min(kFmSB, nblk - ks * kFmSB);
                 for (int h = 0; h < kFmHalves && ok; ++h) {
                     const bool okh = mbar_wait_warp(tfull0 + 8 * h, it & 1, abort_flag);

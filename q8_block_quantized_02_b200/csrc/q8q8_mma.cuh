@@ -304,32 +304,39 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         // ------------------------------ producer ------------------------------
         if (lane == 0 && total > 0) {
             const uint64_t pw = policy_evict_first(), px = policy_evict_last();
-            auto issue_w = [&](int it) {
-                const int slot = it % a.stages;
-                const int tile = t0 + it / ksteps;
-                const int b0 = b_lo + (it % ksteps) * kMmaSB;
+            // ring slot/phase and (tile, k step) are carried along: no
+            // division by a runtime value per stage
+            auto issue_w = [&](int slot, int tile, int ks) {
+                const int b0 = b_lo + ks * kMmaSB;
                 const uint32_t st = smem_u32(smem + (size_t)slot * kMmaStageBytes);
                 const uint32_t full = full0 + 8 * slot;
                 mbar_arrive_expect_tx(full, kMmaTxBytes);
-                tma_load_3d(st, &tq, full, 0, 2 * b0, kMmaTileGroups * tile, pw);
-                tma_load_3d(st + kMmaDOff, &td, full, 0, b0, kMmaTileGroups * tile, pw);
+                tma_load_3d(st, &tq, full, 0, 2 * b0, kMmaTileGroups * (t0 + tile), pw);
+                tma_load_3d(st + kMmaDOff, &td, full, 0, b0, kMmaTileGroups * (t0 + tile), pw);
             };
-            auto issue_x = [&](int it) {
-                const int slot = it % a.stages;
-                const int b0 = b_lo + (it % ksteps) * kMmaSB;
+            auto issue_x = [&](int slot, int ks) {
+                const int b0 = b_lo + ks * kMmaSB;
                 const uint32_t st = smem_u32(smem + (size_t)slot * kMmaStageBytes);
                 tma_load_3d(st + kMmaXOff, &tx, full0 + 8 * slot, 0, 0, 2 * b0, px);
             };
             const int pro = total < a.stages ? total : a.stages;
-            int it = 0;
-            for (; it < pro; ++it) issue_w(it);  // weights never depend on the previous grid
-            pdl_wait_and_trigger();              // activations may
-            for (int k = 0; k < pro; ++k) issue_x(k);
+            int it = 0, tile = 0, ks = 0;
+            for (; it < pro; ++it) {  // weights never depend on the previous grid
+                issue_w(it, tile, ks);
+                if (++ks == ksteps) { ks = 0; ++tile; }
+            }
+            pdl_wait_and_trigger();  // activations may
+            for (int k = 0, kx = 0; k < pro; ++k) {
+                issue_x(k, kx);
+                if (++kx == ksteps) kx = 0;
+            }
+            int slot = pro % a.stages, phase = pro / a.stages;  // ring position of iteration `pro`
             for (; it < total; ++it) {
-                const int slot = it % a.stages;
-                if (!mbar_wait(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag)) break;
-                issue_w(it);
-                issue_x(it);
+                if (!mbar_wait(empty0 + 8 * slot, (phase & 1) ^ 1, abort_flag)) break;
+                issue_w(slot, tile, ks);
+                issue_x(slot, ks);
+                if (++ks == ksteps) { ks = 0; ++tile; }
+                if (++slot == a.stages) { slot = 0; ++phase; }
             }
             *issued = it;
         } else {
@@ -342,11 +349,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
             // Block j of every stage goes to TMEM columns 16 j; the two halves
             // (blocks 0-3, 4-7) are each handed to the epilogue by one commit.
             bool ok = true;
-            for (int it = 0; it < total && ok; ++it) {
-                const int slot = it % a.stages;
-                if (!mbar_wait(full0 + 8 * slot, (it / a.stages) & 1, abort_flag)) break;
+            int slot = 0, phase = 0, ks = 0;  // ring position and k step of iteration `it`
+            for (int it = 0; it < total && ok;
+                 ++it, ks = ks + 1 == ksteps ? 0 : ks + 1, slot = slot + 1 == a.stages ? 0 : slot + 1,
+                     phase ^= slot == 0 ? 1 : 0) {
+                if (!mbar_wait(full0 + 8 * slot, phase, abort_flag)) break;
                 tc_fence_after();
-                const int nb = min(kMmaSB, nblk - (it % ksteps) * kMmaSB);
+                const int nb = min(kMmaSB, nblk - ks * kMmaSB);
                 const uint32_t st = smem_u32(smem + (size_t)slot * kMmaStageBytes);
                 for (int h = 0; h < kMmaHalves; ++h) {
                     // the epilogue has read this half of the previous stage
@@ -388,13 +397,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         const int jt = (e >> 4) & (kMmaSB - 1), nt = e & 15;  // (block in stage, activation row)
         const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + n0;
         pdl_wait_and_trigger();  // activation scales and outputs belong to the previous grid until now
-        auto dx_load = [&](int it) -> float {
+        auto dx_load = [&](int it, int ks) -> float {  // ks: the k step of iteration it
             if (it >= total || !tab_thread) return 0.f;
-            const int b = b_lo + (it % ksteps) * kMmaSB + jt;
+            const int b = b_lo + ks * kMmaSB + jt;
             return (b < b_hi && nt < a.N) ? __half2float(__ushort_as_half(__ldg(a.xd + (size_t)nt * a.B + b)))
                                           : 0.f;
         };
-        float dx_next = dx_load(0);
+        float dx_next = dx_load(0, 0);
         uint64_t acc2[kMmaNPG / 2];  // fp32 pairs (n0 + 2p, n0 + 2p + 1)
         // acc += float(dot) * d_w * d_x for blocks j0 .. j0 + 3 of the stage
         auto compute_half = [&](auto full, const uint32_t(&v)[kMmaHalfBlocks * kMmaNPG], int j0, int nb,
@@ -426,16 +435,16 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                 }
             }
         };
-        int it = 0;
+        int it = 0, slot = 0, phase = 0;  // ring position of iteration `it`, carried along
         for (int tl = 0; tl < n_tiles; ++tl) {
 #pragma unroll
             for (int p = 0; p < kMmaNPG / 2; ++p) acc2[p] = 0ull;
-            for (int ks = 0; ks < ksteps; ++ks, ++it) {
-                const int slot = it % a.stages;
+            for (int ks = 0; ks < ksteps;
+                 ++ks, ++it, slot = slot + 1 == a.stages ? 0 : slot + 1, phase ^= slot == 0 ? 1 : 0) {
                 uint8_t *st = smem + (size_t)slot * kMmaStageBytes;
-                const bool ok = mbar_wait_warp(full0 + 8 * slot, (it / a.stages) & 1, abort_flag);
+                const bool ok = mbar_wait_warp(full0 + 8 * slot, phase, abort_flag);
                 const float dx_cur = dx_next;
-                dx_next = dx_load(it + 1);  // one stage ahead: the load has a stage to land
+                dx_next = dx_load(it + 1, ks + 1 == ksteps ? 0 : ks + 1);  // one stage ahead: it has a stage to land
                 if (ok && tab_thread) {
                     // table entry (jt, nt): d_x and the int bits that fold the
                     // 128 * sum(xq) correction into the float conversion
