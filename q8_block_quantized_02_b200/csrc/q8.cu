@@ -598,6 +598,17 @@ static cudaError_t setup_moe_kernels(int max_smem) {
 }
 static RegisterSetup g_reg_moe(setup_moe_kernels);
 
+static cudaError_t setup_q4k_kernels(int max_smem) {
+    const void *ks[2] = {reinterpret_cast<const void *>(&q4k_tile_kernel<1>),
+                         reinterpret_cast<const void *>(&q4k_tile_kernel<2>)};
+    for (const void *k : ks) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+static RegisterSetup g_reg_q4k(setup_q4k_kernels);
+
 struct MoePlan {
     MoeArgs a;
     size_t smem;
@@ -796,10 +807,17 @@ static q8_status run_kquant(const void *W, const float *x, float *y, int64_t M, 
     if (reinterpret_cast<uintptr_t>(y) & 3u) return Q8_ERR_ALIGN;
     const DeviceInfo *dev = nullptr;
     Q8_CHECK(device_info(&dev));
-    const int64_t warps = std::min<int64_t>(M, (int64_t)dev->sms * 64);
-    const unsigned grid = (unsigned)ceil_div(warps, kKqThreads / 32);
     const int nm = (int)N;
     const uint8_t *w8 = static_cast<const uint8_t *>(W);
+    if (FMT == 4 && N <= 2) {
+        // row tiles, activations in registers (kquant.cuh): about 4 tiles a CTA at least
+        const int64_t tiles = ceil_div(M, kQ4Rows);
+        const unsigned g = (unsigned)std::min<int64_t>(tiles, (int64_t)dev->sms * (N == 1 ? 2 : 1));
+        return N == 1 ? launch_pdl(q4k_tile_kernel<1>, dim3(g), dim3(kQ4Threads), kQ4SmemBytes, stream, name, w8, x, y, (int)M, (int)K, nm)
+                      : launch_pdl(q4k_tile_kernel<2>, dim3(g), dim3(kQ4Threads), kQ4SmemBytes, stream, name, w8, x, y, (int)M, (int)K, nm);
+    }
+    const int64_t warps = std::min<int64_t>(M, (int64_t)dev->sms * 64);
+    const unsigned grid = (unsigned)ceil_div(warps, kKqThreads / 32);
     switch (nmax_for(N)) {
         case 1: return launch_pdl(kquant_gemv_kernel<1, FMT>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
         case 2: return launch_pdl(kquant_gemv_kernel<2, FMT>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);

@@ -35,7 +35,10 @@ def run(fmt, blocks, x, M, K):
 
 @pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
 @pytest.mark.parametrize("M,K,N", [(1, 256, 1), (13, 512, 2), (1000, 3584, 4), (37, 2048, 3),
-                                   (3584, 18944, 1), (4096, 3584, 2)])
+                                   (3584, 18944, 1), (4096, 3584, 2),
+                                   # Q4_K at N <= 2 runs the row-tile kernel: tiles of 32
+                                   # rows (ragged last tile), blocks split over 8 warps
+                                   (33, 256, 1), (4739, 2304, 1), (70, 4864, 2), (5000, 1024, 2)])
 def test_kquant_gemv_matches_oracle(fmt, M, K, N):
     blocks = q8gen.kquant_matrix(fmt, 5 * M + K + N, M, K)
     x = q8gen.activations(M + 2 * K + N, N, K)
@@ -74,3 +77,26 @@ def test_kquant_deterministic_and_rejections():
     with pytest.raises(q8().Q8Error) as e:
         q8().q8_q6k_gemv(w, dev(np.zeros((5, K), np.float32)), y, M, K, 5)    # N > 4
     assert e.value.status == 5
+
+
+@pytest.mark.parametrize("N", [1, 2, 4])
+def test_q4k_zero_weight_sub_blocks(N):
+    """Sub-blocks whose weights are all exactly zero (every nibble q with
+    d*sc*q = dmin*m) contribute nothing: sum |w x| then sees only the other
+    sub-blocks, so a kernel whose rounding scaled with d*sc*sum(q x) or
+    dmin*m*sum(x) instead of with each weight would miss the bar here."""
+    M, K = 300, 1024
+    rng = np.random.default_rng(17)
+    blocks = q8gen.kquant_matrix("q4_k", 19, M, K).reshape(M, K // 256, 144).copy()
+    # d = dmin = 1.0 (binary16 0x3C00); sub-block 0: scale 4, min 12 and every
+    # nibble 3, so w = 4 * 3 - 12 = 0 exactly; sub-blocks 1-7 keep random codes
+    blocks[:, :, 0:2] = np.frombuffer(np.uint16(0x3C00).tobytes(), np.uint8)
+    blocks[:, :, 2:4] = np.frombuffer(np.uint16(0x3C00).tobytes(), np.uint8)
+    blocks[:, :, 4] = (blocks[:, :, 4] & 0xC0) | 4          # sc of sub-block 0
+    blocks[:, :, 8] = (blocks[:, :, 8] & 0xC0) | 12         # m of sub-block 0
+    blocks[:, :, 16:48] = (blocks[:, :, 16:48] & 0xF0) | 3  # low nibbles of bytes 0..31: sub-block 0
+    x = (rng.standard_normal((N, K)) * 10).astype(np.float32)
+    flat = blocks.reshape(-1)
+    y = run("q4_k", flat, x, M, K)
+    y_ref, y_abs = oracle.kquant_gemv("q4_k", flat, x, M, K, threads=oracle.max_threads())
+    assert_within(y, y_ref, TOL_REL * y_abs, f"q4_k zero-weight sub-blocks N={N}")
