@@ -520,9 +520,23 @@ found:
 // (token entries past cnt repeat token cnt - 1, never stored).  Up to two
 // tokens' activations stay in registers for all pieces; more tokens go four
 // at a time, each piece dequantised once per four tokens.
+// Position in the stage ring: the stage count `it`, its slot and the phase
+// parity, carried along (a division by the runtime slot count per stage
+// costs tens of instructions).
+struct MoeRing {
+    int it = 0, slot = 0, phase = 0;
+    __device__ __forceinline__ void next(int stages) {
+        ++it;
+        if (++slot == stages) {
+            slot = 0;
+            phase ^= 1;
+        }
+    }
+};
+
 template <int PH, int NX, int CW, bool FULL>
 __device__ __forceinline__ void moe_consume(const uint8_t *smem, const MoeArgs &a, uint32_t full0,
-                                            uint32_t empty0, volatile int *abort_flag, int &it,
+                                            uint32_t empty0, volatile int *abort_flag, MoeRing &it,
                                             const MoeTile &t, int quad, int hf, int lane,
                                             float (&acc)[(moe_tg(PH, NX) / (CW / 8)) * moe_halves(PH)][NX]) {
     constexpr int HH = moe_halves(PH), TG = moe_tg(PH, NX), TGH = TG / (CW / 8), NP = TGH * HH;
@@ -542,9 +556,9 @@ __device__ __forceinline__ void moe_consume(const uint8_t *smem, const MoeArgs &
     for (int p = 0; p < NP; ++p)
 #pragma unroll
         for (int n = 0; n < NX; ++n) acc[p][n] = 0.f;
-    for (int ks = 0; ks < t.ks_n; ++ks, ++it) {
-        const int slot = it % a.stages;
-        if (mbar_wait_warp(full0 + 8 * slot, (it / a.stages) & 1, abort_flag)) {
+    for (int ks = 0; ks < t.ks_n; ++ks, it.next(a.stages)) {
+        const int slot = it.slot;
+        if (mbar_wait_warp(full0 + 8 * slot, it.phase, abort_flag)) {
             const uint8_t *st = smem + (size_t)slot * a.slot_bytes;
             const int cols = min(kMoeCS, t.cols - ks * kMoeCS);
             if (col < cols && any) {
@@ -624,7 +638,7 @@ __device__ __forceinline__ void moe_consume(const uint8_t *smem, const MoeArgs &
 template <int PH, int NX, int CW>
 __device__ __forceinline__ void moe_consume_tile(const uint8_t *smem, const MoeArgs &a, uint32_t full0,
                                                  uint32_t empty0, uint32_t redfull0, uint32_t redfree0,
-                                                 float *red, volatile int *abort_flag, int &it, int tl,
+                                                 float *red, volatile int *abort_flag, MoeRing &it, int tl,
                                                  const MoeTile &t, int quad, int hf, int lane) {
     constexpr int HH = moe_halves(PH), TGH = moe_tg(PH, NX) / (CW / 8), NP = TGH * HH;
     float acc[NP][NX];
@@ -650,7 +664,7 @@ __device__ __forceinline__ void moe_consume_tile(const uint8_t *smem, const MoeA
 template <int PH, int NMAX, int CW>
 __device__ __forceinline__ void moe_consume_any(const uint8_t *smem, const MoeArgs &a, uint32_t full0,
                                                 uint32_t empty0, uint32_t redfull0, uint32_t redfree0,
-                                                float *red, volatile int *abort_flag, int &it, int tl,
+                                                float *red, volatile int *abort_flag, MoeRing &it, int tl,
                                                 const MoeTile &t, int quad, int hf, int lane) {
 #define Q8_MOE_TILE(NXV)                                                                                  \
     moe_consume_tile<PH, (NXV < NMAX ? NXV : NMAX), CW>(smem, a, full0, empty0, redfull0, redfree0, red,     \
@@ -827,7 +841,7 @@ struct MoeMaps {
 // Returns false (warp-uniform) when a wait failed.
 __device__ __forceinline__ bool moe_issue_weights(uint8_t *smem, const MoeArgs &a, const MoeMaps &m,
                                                   const MoeTable &tb, uint32_t full0, uint32_t empty0,
-                                                  volatile int *abort_flag, int &it, const MoeTile &t,
+                                                  volatile int *abort_flag, MoeRing &it, const MoeTile &t,
                                                   uint64_t pw, int lane) {
     const int HH = t.phase == 1 ? 2 : 1, TG = moe_tg(t.phase, t.nx);
     const bool shared = t.seg < 0;
@@ -843,9 +857,9 @@ __device__ __forceinline__ bool moe_issue_weights(uint8_t *smem, const MoeArgs &
     const CUtensorMap(&maps)[2][kMoeDepths] = m.w[t.phase - 1][shared ? 1 : 0];
     const int bits = __popc(t.tga), per = bits * HH;  // boxes per half, per stage (q; scales alike)
     const uint32_t dbase = (uint32_t)HH * TG * kMoeQBox;
-    for (int ks = 0; ks < t.ks_n; ++ks, ++it) {
-        const int slot = it % a.stages;
-        if (it >= a.stages && !mbar_wait_warp(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag))
+    for (int ks = 0; ks < t.ks_n; ++ks, it.next(a.stages)) {
+        const int slot = it.slot;
+        if (it.it >= a.stages && !mbar_wait_warp(empty0 + 8 * slot, it.phase ^ 1, abort_flag))
             return false;
         const uint32_t st = smem_u32(smem + (size_t)slot * a.slot_bytes);
         const uint32_t full = full0 + 8 * slot;
@@ -876,7 +890,7 @@ __device__ __forceinline__ bool moe_issue_weights(uint8_t *smem, const MoeArgs &
 // complete).  Returns false when a wait failed.
 __device__ __forceinline__ bool moe_issue_acts(uint8_t *smem, const MoeArgs &a, const MoeMaps &m,
                                                const MoeTable &tb, uint32_t full0, uint32_t empty0,
-                                               volatile int *abort_flag, int &it, const MoeTile &t,
+                                               volatile int *abort_flag, MoeRing &it, const MoeTile &t,
                                                uint64_t px) {
     const bool shared = t.seg < 0;
     if (t.phase == 2) {
@@ -887,9 +901,9 @@ __device__ __forceinline__ bool moe_issue_acts(uint8_t *smem, const MoeArgs &a, 
     }
     const uint32_t xoff = moe_x_off(t.phase, t.nx);
     const int row0 = shared ? 0 : tb.seg_row0[t.seg];
-    for (int ks = 0; ks < t.ks_n; ++ks, ++it) {
-        const int slot = it % a.stages;
-        if (it >= a.stages && !mbar_wait(empty0 + 8 * slot, ((it / a.stages) & 1) ^ 1, abort_flag)) return false;
+    for (int ks = 0; ks < t.ks_n; ++ks, it.next(a.stages)) {
+        const int slot = it.slot;
+        if (it.it >= a.stages && !mbar_wait(empty0 + 8 * slot, it.phase ^ 1, abort_flag)) return false;
         const uint32_t st = smem_u32(smem + (size_t)slot * a.slot_bytes) + xoff;
         const uint32_t full = full0 + 8 * slot;
         mbar_arrive_expect_tx(full, (uint32_t)t.cnt * kMoeXRow);
@@ -952,7 +966,7 @@ __global__ void __launch_bounds__(moe_threads(NMAX), 1)
         // ------------------------- weight producer -------------------------
         {
             const uint64_t pw = policy_evict_first();
-            int it = 0;
+            MoeRing it;
             bool ok = true;
             // the shared expert's gate|up boxes need nothing from earlier kernels
             while (ok && moe_next(cur, rg, tb, a, t))
@@ -963,14 +977,14 @@ __global__ void __launch_bounds__(moe_threads(NMAX), 1)
                 while (ok && moe_next(cur, rg, tb, a, t))
                     ok = moe_issue_weights(smem, a, maps, tb, full0, empty0, abort_flag, it, t, pw, lane);
             }
-            if (lane == 0) *issued_w = it;
+            if (lane == 0) *issued_w = it.it;
         }
     } else if (warp == CW + 1) {
         // ----------------------- activation producer -----------------------
         pdl_wait_and_trigger();  // x comes from the previous kernel
         if (lane == 0) {
             const uint64_t px = policy_evict_last();
-            int it = 0;
+            MoeRing it;
             bool ok = true;
             while (ok && moe_next(cur, rg, tb, a, t)) ok = moe_issue_acts(smem, a, maps, tb, full0, empty0, abort_flag, it, t, px);
             if (ok && mbar_wait(tbl_ready, 0, abort_flag)) {
@@ -978,7 +992,7 @@ __global__ void __launch_bounds__(moe_threads(NMAX), 1)
                 while (ok && moe_next(cur, rg, tb, a, t))
                     ok = moe_issue_acts(smem, a, maps, tb, full0, empty0, abort_flag, it, t, px);
             }
-            *issued_x = it;
+            *issued_x = it.it;
         }
     } else if (warp == CW + 2) {
         // ------------------------ table + epilogues ------------------------
@@ -1013,7 +1027,8 @@ __global__ void __launch_bounds__(moe_threads(NMAX), 1)
         // ----------------------------- consumers ----------------------------
         const int quad = warp & 7, hf = warp >> 3;
         pdl_wait_and_trigger();
-        int it = 0, tl = 0;
+        MoeRing it;
+        int tl = 0;
         for (;;) {
             if (!moe_next(cur, rg, tb, a, t)) {
                 if (rg.table || !mbar_wait_warp(tbl_ready, 0, abort_flag)) break;

@@ -985,8 +985,9 @@ q8_status q8_quantize_act(const float *x, int8_t *xq, uint16_t *xd, int64_t N, i
     if (reinterpret_cast<uintptr_t>(xd) & 1u) return Q8_ERR_ALIGN;
     const DeviceInfo *dev = nullptr;
     Q8_CHECK(device_info(&dev));
-    const int64_t blocks = std::min<int64_t>(ceil_div(N * (K / 32), 128), (int64_t)dev->sms * 8);
-    return launch_pdl(quantize_act_kernel, dim3((unsigned)blocks), dim3(128), 0,
+    // a warp per 32-block, 8 warps a CTA
+    const int64_t blocks = std::min<int64_t>(ceil_div(N * (K / 32), 8), (int64_t)dev->sms * 8);
+    return launch_pdl(quantize_act_kernel, dim3((unsigned)blocks), dim3(256), 0,
                       (cudaStream_t)stream, "q8_quantize_act launch", x, xq, xd, N, K);
 }
 

@@ -7,63 +7,37 @@
 
 namespace q8 {
 
-// One thread per (row n, block b): amax over the block, d32 = amax / 127,
+// Per (row n, block b), one warp: amax over the block, d32 = amax / 127,
 // q = roundf(x / d32) clamped to +-127 (roundf rounds half away from zero),
 // stored scale = binary16 RN of d32.  Divisions are IEEE round-to-nearest
 // (__fdiv_rn) so the result is bit-exact with any IEEE implementation of the
 // same steps.
 __global__ void quantize_act_kernel(const float *__restrict__ x, int8_t *__restrict__ xq,
                                     uint16_t *__restrict__ xd, int64_t N, int64_t K) {
+    // one warp per 32-block, lane i takes element i (the loads of a warp are
+    // one coalesced 128-byte line; the block's max by a shuffle tree, exact)
     pdl_wait();
     pdl_launch_dependents();
     const int64_t B = K / 32;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N * B;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const float4 *src = reinterpret_cast<const float4 *>(x + i * 32);
-        float v[32];
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t i = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); i < N * B; i += warps) {
+        const float v = x[i * 32 + lane];
+        float amax = fabsf(v);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const float4 f = src[k];
-            v[4 * k] = f.x;
-            v[4 * k + 1] = f.y;
-            v[4 * k + 2] = f.z;
-            v[4 * k + 3] = f.w;
-        }
-        float amax = 0.0f;
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const float a = fabsf(v[k]);
-            if (a > amax) amax = a;
-        }
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         const float d32 = __fdiv_rn(amax, 127.0f);
-        uint32_t packed[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                int q = 0;
-                if (d32 != 0.0f) {
-                    float r = roundf(__fdiv_rn(v[4 * k + b], d32));
-                    r = fminf(fmaxf(r, -127.0f), 127.0f);
-                    q = (int)r;
-                }
-                word |= ((uint32_t)(q & 0xff)) << (8 * b);
-            }
-            packed[k] = word;
+        int q = 0;
+        if (d32 != 0.0f) {
+            float r = roundf(__fdiv_rn(v, d32));
+            r = fminf(fmaxf(r, -127.0f), 127.0f);
+            q = (int)r;
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(xq + i * 32);
-        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-        xd[i] = __half_as_ushort(__float2half_rn(d32));
+        xq[i * 32 + lane] = (int8_t)q;
+        if (lane == 0) xd[i] = __half_as_ushort(__float2half_rn(d32));
     }
 }
 
-// RMSNorm in front of the quantiser (the norm that precedes every Qwen
-// projection: "augur" README, "Features"), one CTA per activation row so the
-// sum of squares never leaves the CTA (the cross-work-group reduction race of
-// "Add Qwen1.5-MoE Q8_0 ... - #144", conversation): fp32 squares summed
-// per thread with FMA, then across lanes and warps in a fixed order;
 // r = 1 / sqrt(sum / K + eps), correctly rounded; xhat = (x * r) * gamma, two
 // fp32 roundings in that order (the "augur" README's Triton RMSNorm, section
 // "Kernels", sums in fp32 and keeps its reference's order of conversions);
