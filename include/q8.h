@@ -207,7 +207,8 @@ static inline float q8_argmax_value(uint64_t key) {
  * blocks).  W: [M][K/256] blocks, rows contiguous, unpacked.  x: [N][K] fp32,
  * 16-byte aligned.  y: [N][M] fp32.  K % 256 == 0; 1 <= N <= 4.  Each output
  * is within 1e-5 * sum_k |w x| of the exact value (every weight formed with
- * at most one fp32 rounding).  CUDA cores, one warp per row.
+ * at most one fp32 rounding).  CUDA cores: Q4_K at N <= 2 in tiles of 32 rows
+ * fed by TMA boxes, otherwise one warp per row.
  * Q4_K, 144-byte blocks, W 16-byte aligned: d (binary16) | dmin (binary16) |
  *   scales[12] | qs[128].  Sub-block j (weights 32j..32j+31) has a 6-bit
  *   scale sc and min m: j < 4: sc = scales[j] & 63, m = scales[j+4] & 63;
@@ -222,6 +223,28 @@ q8_status q8_q4k_gemv(const void *W, const float *x, float *y, int64_t M, int64_
                       q8_stream_t stream);
 q8_status q8_q6k_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
                       q8_stream_t stream);
+
+/* Q6_K packed for the tile kernel.  Raw 210-byte blocks start on 2-byte
+ * boundaries, which TMA and 16-byte copies cannot fetch, so the blocks are
+ * re-laid once into 6720-byte units, one per (tile of 32 rows, block):
+ *   unit (t, b) at byte (t * (K/256) + b) * 6720; row i of the tile (matrix
+ *   row 32t + i) at byte 208 i of the unit holds bytes 0..207 of its raw
+ *   block b (ql | qh | scales); bytes 6656 + 2i and 6657 + 2i hold its d;
+ *   rows past M are zero.
+ * q8_q6k_packed_bytes: ceil(M/32) * (K/256) * 6720 (0 for a bad shape).
+ * q8_q6k_pack_weights: raw (device, [M][K/256] blocks, any alignment) ->
+ *   packed (device, 16-byte aligned, fully written).  q8_q6k_unpack_weights:
+ *   the inverse (bit-exact round trip).  q8_q6k_gemv_packed: the product of
+ *   q8_q6k_gemv from the packed units, same arguments, bound and N <= 4
+ *   (activation rows two per launch); each 16-weight run is summed as
+ *   sum (q - 32) x and scaled once by d * scale (exact), so the bound is
+ *   unchanged.  Shape and pointer errors are reported before anything is
+ *   enqueued. */
+size_t q8_q6k_packed_bytes(int64_t M, int64_t K);
+q8_status q8_q6k_pack_weights(const void *raw, int64_t M, int64_t K, void *packed, q8_stream_t stream);
+q8_status q8_q6k_unpack_weights(const void *packed, int64_t M, int64_t K, void *raw, q8_stream_t stream);
+q8_status q8_q6k_gemv_packed(const void *packed, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                             q8_stream_t stream);
 
 /* ---------------------------------------------------------------------- */
 /* S4  Fused gate_up + SwiGLU                                              */

@@ -21,6 +21,7 @@ __all__ = [
     "q8_version", "q8_packed_bytes", "q8_pack_weights", "q8_unpack_weights", "q8_gemv",
     "q8_gemv_residual", "q8_gemv_argmax", "q8_argmax_index", "q8_argmax_value",
     "q8_q4k_gemv", "q8_q6k_gemv",
+    "q8_q6k_packed_bytes", "q8_q6k_pack_weights", "q8_q6k_unpack_weights", "q8_q6k_gemv_packed",
     "q8_gate_up_swiglu", "q8_moe_route", "q8_moe_workspace_bytes", "q8_moe_workspace_init",
     "q8_moe_gemv",
     "q8_moe_gemv_noalloc",
@@ -51,6 +52,10 @@ _SIGS = {
     "q8_gemv_residual": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "q8_q4k_gemv": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "q8_q6k_gemv": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
+    "q8_q6k_packed_bytes": (_SZ, [_I64, _I64]),
+    "q8_q6k_pack_weights": (_INT, [_P, _I64, _I64, _P, _P]),
+    "q8_q6k_unpack_weights": (_INT, [_P, _I64, _I64, _P, _P]),
+    "q8_q6k_gemv_packed": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "q8_gate_up_swiglu": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "q8_moe_route": (_INT, [_P, _I64, _I64, _I64, _INT, _P, _P, _P]),
     "q8_moe_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I64, _I64, _I64]),
@@ -169,6 +174,24 @@ def q8_q4k_gemv(W, x, y, M, K, N, stream=None):
 def q8_q6k_gemv(W, x, y, M, K, N, stream=None):
     """W: raw GGUF Q6_K blocks (uint8 device tensor)."""
     _call("q8_q6k_gemv", _ptr(W), _ptr(x), _ptr(y), M, K, N, _stream(stream))
+
+
+def q8_q6k_packed_bytes(M: int, K: int) -> int:
+    return int(_load().q8_q6k_packed_bytes(M, K))
+
+
+def q8_q6k_pack_weights(raw, M, K, packed, stream=None):
+    """raw GGUF Q6_K blocks -> the tile kernel's 6720-byte units."""
+    _call("q8_q6k_pack_weights", _ptr(raw), M, K, _ptr(packed), _stream(stream))
+
+
+def q8_q6k_unpack_weights(packed, M, K, raw, stream=None):
+    _call("q8_q6k_unpack_weights", _ptr(packed), M, K, _ptr(raw), _stream(stream))
+
+
+def q8_q6k_gemv_packed(packed, x, y, M, K, N, stream=None):
+    """packed: q8_q6k_pack_weights output (uint8 device tensor)."""
+    _call("q8_q6k_gemv_packed", _ptr(packed), _ptr(x), _ptr(y), M, K, N, _stream(stream))
 
 
 def q8_gemv_residual(W, x, residual, y, M, K, N, stream=None):

@@ -244,6 +244,51 @@ inline q8_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
     return launch_pdl_cluster(kernel, grid, block, smem, stream, name, 1u, std::forward<Args>(args)...);
 }
 
+// How many clusters of `cluster_x` CTAs of `kernel` (threads, dynamic shared
+// memory) the current device runs at once; cached per (device, kernel,
+// threads, smem, cluster size).  Clusters are placed within one GPC, so with
+// one CTA per SM a cluster size that does not divide a GPC's SMs leaves SMs
+// idle: 28 clusters of 5 do not fit at once on a 148-SM part (26 do), and the
+// last ones would run as a second wave.  0 when the query fails.
+inline int max_active_clusters(const void *kernel, int threads, size_t smem, int cluster_x) {
+    struct Entry {
+        int dev;
+        const void *k;
+        int threads;
+        size_t smem;
+        int cx;
+        int n;
+    };
+    static Entry cache[64];
+    static int used = 0;
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+        if (cache[i].dev == dev && cache[i].k == kernel && cache[i].threads == threads && cache[i].smem == smem &&
+            cache[i].cx == cluster_x)
+            return cache[i].n;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cluster_x);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster_x;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();  // not sticky; clear it
+        return 0;
+    }
+    if (used < 64) cache[used++] = Entry{dev, kernel, threads, smem, cluster_x, n};
+    return n;
+}
+
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 

@@ -429,30 +429,38 @@ struct MmaPlan {
 
 // One CTA per SM.  With at least as many 128-row tiles as SMs each cluster is
 // one CTA walking a contiguous tile range; with fewer, every tile gets a
-// cluster of up to 8 CTAs that split K between them.
+// cluster of up to 8 CTAs that split K between them: the largest split whose
+// clusters all run at once (max_active_clusters), else none.
 static MmaPlan plan_mma(int64_t M, int64_t K, int64_t N, int sms) {
     MmaPlan p;
     MmaArgs &a = p.a;
     a = MmaArgs{};
     const int64_t B = K / 32;
     const int64_t tiles = ceil_div(ceil_div(M, kGroupRows), kMmaTileGroups);
-    int64_t split = 1, clusters = sms;
-    if (tiles < sms) {
-        split = std::min<int64_t>(kMmaMaxSplit, sms / tiles);
-        split = std::min<int64_t>(split, B);  // every CTA keeps at least one block
-        if (split < 1) split = 1;
-        clusters = tiles;
-    }
-    const int64_t blocks = ceil_div(B, split);
-    const int64_t per_cta = ceil_div(tiles, clusters) * ceil_div(blocks, kMmaSB);
     a.M = (int)M;
     a.N = (int)N;
     a.B = (int)B;
     a.tiles = (int)tiles;
-    a.split = (int)split;
-    a.stages = (int)std::max<int64_t>(1, std::min<int64_t>(kMmaMaxStages, per_cta));
-    p.grid = (int)(clusters * split);
-    p.smem = mma_smem_bytes(a.stages, split > 1);
+    auto finish = [&](int64_t split) {
+        const int64_t clusters = tiles < sms ? tiles : sms;
+        const int64_t blocks = ceil_div(B, split);
+        const int64_t per_cta = ceil_div(tiles, clusters) * ceil_div(blocks, kMmaSB);
+        a.split = (int)split;
+        a.stages = (int)std::max<int64_t>(1, std::min<int64_t>(kMmaMaxStages, per_cta));
+        p.grid = (int)(clusters * split);
+        p.smem = mma_smem_bytes(a.stages, split > 1);
+    };
+    int64_t split = 1;
+    if (tiles < sms) {
+        split = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(kMmaMaxSplit, sms / tiles), B));
+        for (; split > 1; --split) {
+            finish(split);
+            if (max_active_clusters(reinterpret_cast<const void *>(&q8q8_mma_kernel), kMmaThreads, p.smem,
+                                    (int)split) >= tiles)
+                break;
+        }
+    }
+    finish(split);
     return p;
 }
 
@@ -512,31 +520,37 @@ struct FmPlan {
 // One CTA per SM.  A tile is 128 output rows (SwiGLU: 64 outputs, their gate
 // and up rows).  With at least as many tiles as SMs each cluster is one CTA
 // walking a contiguous tile range; with fewer, every tile gets a cluster of up
-// to 8 CTAs that split K between them.
-static FmPlan plan_fm(int64_t rows_out, int64_t K, int64_t N, bool swiglu, int sms) {
+// to 8 CTAs that split K between them: the largest split whose clusters all
+// run at once (max_active_clusters of `kern`), else none.
+static FmPlan plan_fm(int64_t rows_out, int64_t K, int64_t N, bool swiglu, int sms, const void *kern) {
     FmPlan p;
     FmArgs &a = p.a;
     a = FmArgs{};
     const int64_t B = K / 32;
     const int64_t tiles = ceil_div(rows_out, swiglu ? 64 : 128);
-    int64_t split = 1, clusters = sms;
-    if (tiles < sms) {
-        split = std::min<int64_t>(kFmMaxSplit, sms / tiles);
-        split = std::min<int64_t>(split, B);  // every CTA keeps at least one block
-        if (split < 1) split = 1;
-        clusters = tiles;
-    }
-    const int64_t blocks = ceil_div(B, split);
-    const int64_t per_cta = ceil_div(tiles, clusters) * ceil_div(blocks, kFmSB);
     a.M_out = (int)rows_out;
     a.N = (int)N;
     a.B = (int)B;
     a.tiles = (int)tiles;
-    a.split = (int)split;
-    a.stages = (int)std::max<int64_t>(1, std::min<int64_t>(kFmMaxStages, per_cta));
     a.up_group0 = swiglu ? (int)(rows_out / kGroupRows) : 0;
-    p.grid = (int)(clusters * split);
-    p.smem = fm_smem_bytes(a.stages);
+    auto finish = [&](int64_t split) {
+        const int64_t clusters = tiles < sms ? tiles : sms;
+        const int64_t blocks = ceil_div(B, split);
+        const int64_t per_cta = ceil_div(tiles, clusters) * ceil_div(blocks, kFmSB);
+        a.split = (int)split;
+        a.stages = (int)std::max<int64_t>(1, std::min<int64_t>(kFmMaxStages, per_cta));
+        p.grid = (int)(clusters * split);
+        p.smem = fm_smem_bytes(a.stages);
+    };
+    int64_t split = 1;
+    if (tiles < sms) {
+        split = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(kFmMaxSplit, sms / tiles), B));
+        for (; split > 1; --split) {
+            finish(split);
+            if (max_active_clusters(kern, kFmThreads, p.smem, (int)split) >= tiles) break;
+        }
+    }
+    finish(split);
     return p;
 }
 
@@ -547,7 +561,11 @@ static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_ou
     const int64_t B = K / 32, C = K / 16;
     const int64_t units = ceil_div(rows_out, kGroupRows);
     const int64_t groups = swiglu ? 2 * units : units;
-    FmPlan p = plan_fm(rows_out, K, N, swiglu, dev->sms);
+    using FmKernel = void (*)(CUtensorMap, CUtensorMap, const float *, FmArgs);
+    // each epilogue warp takes 1 activation row up to N = 4, 2 up to N = 8, else 4
+    const FmKernel k = swiglu ? (N <= 4 ? &f32_mma_kernel<true, 1> : N <= 8 ? &f32_mma_kernel<true, 2> : &f32_mma_kernel<true, 4>)
+                              : (N <= 4 ? &f32_mma_kernel<false, 1> : N <= 8 ? &f32_mma_kernel<false, 2> : &f32_mma_kernel<false, 4>);
+    FmPlan p = plan_fm(rows_out, K, N, swiglu, dev->sms, reinterpret_cast<const void *>(k));
     if (p.smem > (size_t)dev->max_smem_optin) return Q8_ERR_UNSUPPORTED;
     p.a.y = y;
     p.a.res = swiglu ? nullptr : res;
@@ -560,11 +578,7 @@ static q8_status run_fm(const void *W, const float *x, float *y, int64_t rows_ou
     // scales: [group][block][8 rows] fp16, 8 groups x kFmSB blocks a box
     Q8_CHECK(make_map_3d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT16, dbase, 8, B, groups, 16, gstride, 8,
                          kFmSB, 8, true));
-    // the activations are read by the kernel's splitter warps with plain loads;
-    // each epilogue warp takes 1 activation row up to N = 4, 2 up to N = 8, else 4
-    using FmKernel = void (*)(CUtensorMap, CUtensorMap, const float *, FmArgs);
-    const FmKernel k = swiglu ? (N <= 4 ? &f32_mma_kernel<true, 1> : N <= 8 ? &f32_mma_kernel<true, 2> : &f32_mma_kernel<true, 4>)
-                              : (N <= 4 ? &f32_mma_kernel<false, 1> : N <= 8 ? &f32_mma_kernel<false, 2> : &f32_mma_kernel<false, 4>);
+    // the activations are read by the kernel's splitter warps with plain loads
     return launch_pdl_cluster(k, dim3(p.grid), dim3(kFmThreads), p.smem, stream,
                               swiglu ? "q8_gate_up_swiglu (tensor cores) launch" : "q8_gemv (tensor cores) launch",
                               (unsigned)p.a.split, tq, td, x, p.a);
@@ -598,13 +612,24 @@ static cudaError_t setup_moe_kernels(int max_smem) {
 }
 static RegisterSetup g_reg_moe(setup_moe_kernels);
 
+// K-quant tile kernel variants: (format, N, stages, CTAs per SM).  Two CTAs
+// per SM at N = 1 (twice the warps to hide the dequantise-and-dot latency);
+// at N = 2 the registers allow one, with deeper rings.
+#define Q8_KQ_VARIANTS(X) X(4, 1, 3, 2) X(4, 2, 4, 1) X(6, 1, 2, 2) X(6, 2, 3, 1)
 static cudaError_t setup_q4k_kernels(int max_smem) {
-    const void *ks[2] = {reinterpret_cast<const void *>(&q4k_tile_kernel<1>),
-                         reinterpret_cast<const void *>(&q4k_tile_kernel<2>)};
-    for (const void *k : ks) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-        if (e != cudaSuccess) return e;
+    (void)max_smem;
+#define Q8_KQ_SETUP(F, NM, ST, MB)                                                                             \
+    {                                                                                                        \
+        const void *k = reinterpret_cast<const void *>(&kq_tile_kernel<F, NM, ST, MB>);                      \
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,                 \
+                                             kq_smem_bytes<F, NM, ST>());                                    \
+        if (e != cudaSuccess) return e;                                                                      \
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,                          \
+                                 cudaSharedmemCarveoutMaxShared);                                            \
+        if (e != cudaSuccess) return e;                                                                      \
     }
+    Q8_KQ_VARIANTS(Q8_KQ_SETUP)
+#undef Q8_KQ_SETUP
     return cudaSuccess;
 }
 static RegisterSetup g_reg_q4k(setup_q4k_kernels);
@@ -795,26 +820,48 @@ static q8_status moe_launch(MoePlan &p, const void *gate_up_experts, const void 
                       stream, "q8_moe_gemv launch", m, a);
 }
 
-template <int FMT>
-// K-quant GEMV launch (kquant.cuh): argument checks, then one warp per row.
-static q8_status run_kquant(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
-                            cudaStream_t stream, const char *name) {
+// One launch of the K-quant tile kernel (kquant.cuh) for N <= 2: a CTA per
+// 32-row tile, at most MINB per SM.
+template <int FMT, int NM, int ST, int MB>
+static q8_status launch_kq_tile(const CUtensorMap &map, const uint8_t *w8, const float *x, float *y, int64_t M,
+                                int64_t K, int N, int sms, cudaStream_t stream, const char *name) {
+    const int64_t tiles = ceil_div(M, kKqRows);
+    const unsigned g = (unsigned)std::min<int64_t>(tiles, (int64_t)sms * MB);
+    return launch_pdl(kq_tile_kernel<FMT, NM, ST, MB>, dim3(g), dim3(kKqTileThreads),
+                      (size_t)kq_smem_bytes<FMT, NM, ST>(), stream, name, map, w8, x, y, (int)M, (int)K, N);
+}
+
+// K-quant argument checks shared by the entry points.
+static q8_status kquant_check(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                              bool w_aligned) {
     if (M <= 0 || K <= 0 || N <= 0 || K % 256) return Q8_ERR_SHAPE;
     if (N > 4 || M > (int64_t)1 << 30 || K > (int64_t)1 << 24) return Q8_ERR_UNSUPPORTED;
-    Q8_CHECK(check_device_ptr(W, FMT == 4));  // Q4_K blocks are read as aligned words
+    Q8_CHECK(check_device_ptr(W, w_aligned));
     Q8_CHECK(check_device_ptr(x));
     Q8_CHECK(check_device_ptr(y, false));
     if (reinterpret_cast<uintptr_t>(y) & 3u) return Q8_ERR_ALIGN;
+    return Q8_OK;
+}
+
+template <int FMT>
+// K-quant GEMV on raw blocks: argument checks, then the tile kernel (Q4_K,
+// N <= 2) or one warp per row.
+static q8_status run_kquant(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                            cudaStream_t stream, const char *name) {
+    Q8_CHECK(kquant_check(W, x, y, M, K, N, FMT == 4));  // Q4_K blocks are read as aligned words / TMA boxes
     const DeviceInfo *dev = nullptr;
     Q8_CHECK(device_info(&dev));
     const int nm = (int)N;
     const uint8_t *w8 = static_cast<const uint8_t *>(W);
     if (FMT == 4 && N <= 2) {
-        // row tiles, activations in registers (kquant.cuh): about 4 tiles a CTA at least
-        const int64_t tiles = ceil_div(M, kQ4Rows);
-        const unsigned g = (unsigned)std::min<int64_t>(tiles, (int64_t)dev->sms * (N == 1 ? 2 : 1));
-        return N == 1 ? launch_pdl(q4k_tile_kernel<1>, dim3(g), dim3(kQ4Threads), kQ4SmemBytes, stream, name, w8, x, y, (int)M, (int)K, nm)
-                      : launch_pdl(q4k_tile_kernel<2>, dim3(g), dim3(kQ4Threads), kQ4SmemBytes, stream, name, w8, x, y, (int)M, (int)K, nm);
+        // raw rows of 144 * SB bytes: boxes of {one 144-byte block, 32 rows}
+        const int64_t SB = K / 256;
+        CUtensorMap map;
+        const q8_status ms =
+            make_map_3d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, 144, SB, M, 144, 144 * SB, 144, 1, kKqRows, true);
+        if (ms != Q8_OK) return ms;
+        return N == 1 ? launch_kq_tile<4, 1, 3, 2>(map, w8, x, y, M, K, nm, dev->sms, stream, name)
+                      : launch_kq_tile<4, 2, 4, 1>(map, w8, x, y, M, K, nm, dev->sms, stream, name);
     }
     const int64_t warps = std::min<int64_t>(M, (int64_t)dev->sms * 64);
     const unsigned grid = (unsigned)ceil_div(warps, kKqThreads / 32);
@@ -823,6 +870,27 @@ static q8_status run_kquant(const void *W, const float *x, float *y, int64_t M, 
         case 2: return launch_pdl(kquant_gemv_kernel<2, FMT>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
         default: return launch_pdl(kquant_gemv_kernel<4, FMT>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
     }
+}
+
+// Q6_K on the packed units: the tile kernel, activation rows two at a time.
+static q8_status run_q6k_packed(const void *P, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                                cudaStream_t stream) {
+    Q8_CHECK(kquant_check(P, x, y, M, K, N, true));
+    const DeviceInfo *dev = nullptr;
+    Q8_CHECK(device_info(&dev));
+    const char *name = "q8_q6k_gemv_packed launch";
+    const uint8_t *w8 = static_cast<const uint8_t *>(P);
+    CUtensorMap unused;
+    std::memset(&unused, 0, sizeof(unused));
+    for (int64_t n0 = 0; n0 < N; n0 += 2) {
+        const int nm = (int)std::min<int64_t>(2, N - n0);
+        const float *xn = x + n0 * K;
+        float *yn = y + n0 * M;
+        const q8_status st = nm == 1 ? launch_kq_tile<6, 1, 2, 2>(unused, w8, xn, yn, M, K, 1, dev->sms, stream, name)
+                                     : launch_kq_tile<6, 2, 3, 1>(unused, w8, xn, yn, M, K, 2, dev->sms, stream, name);
+        if (st != Q8_OK) return st;
+    }
+    return Q8_OK;
 }
 
 }  // namespace q8
@@ -923,6 +991,44 @@ q8_status q8_q4k_gemv(const void *W, const float *x, float *y, int64_t M, int64_
 q8_status q8_q6k_gemv(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
                       q8_stream_t stream) {
     return run_kquant<6>(W, x, y, M, K, N, (cudaStream_t)stream, "q8_q6k_gemv launch");
+}
+
+size_t q8_q6k_packed_bytes(int64_t M, int64_t K) {
+    if (M <= 0 || K <= 0 || K % 256) return 0;
+    return (size_t)ceil_div(M, kKqRows) * (size_t)(K / 256) * kQ6UnitBytes;
+}
+
+q8_status q8_q6k_pack_weights(const void *raw, int64_t M, int64_t K, void *packed, q8_stream_t stream) {
+    if (M <= 0 || K <= 0 || K % 256) return Q8_ERR_SHAPE;
+    if (M > (int64_t)1 << 30 || K > (int64_t)1 << 24) return Q8_ERR_UNSUPPORTED;
+    Q8_CHECK(check_device_ptr(raw, false));
+    Q8_CHECK(check_device_ptr(packed));
+    const DeviceInfo *dev = nullptr;
+    Q8_CHECK(device_info(&dev));
+    const long long pieces = (long long)(q8_q6k_packed_bytes(M, K) / 16);
+    const unsigned grid = (unsigned)std::min<long long>((pieces + 255) / 256, (long long)dev->sms * 16);
+    return launch_pdl(q6k_pack_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, "q8_q6k_pack_weights launch",
+                      static_cast<const uint8_t *>(raw), static_cast<uint8_t *>(packed), (int)M, (int)(K / 256),
+                      pieces);
+}
+
+q8_status q8_q6k_unpack_weights(const void *packed, int64_t M, int64_t K, void *raw, q8_stream_t stream) {
+    if (M <= 0 || K <= 0 || K % 256) return Q8_ERR_SHAPE;
+    if (M > (int64_t)1 << 30 || K > (int64_t)1 << 24) return Q8_ERR_UNSUPPORTED;
+    Q8_CHECK(check_device_ptr(packed));
+    Q8_CHECK(check_device_ptr(raw, false));
+    const DeviceInfo *dev = nullptr;
+    Q8_CHECK(device_info(&dev));
+    const long long bytes = (long long)M * (K / 256) * 210;
+    const unsigned grid = (unsigned)std::min<long long>((bytes + 255) / 256, (long long)dev->sms * 16);
+    return launch_pdl(q6k_unpack_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream,
+                      "q8_q6k_unpack_weights launch", static_cast<const uint8_t *>(packed),
+                      static_cast<uint8_t *>(raw), (int)M, (int)(K / 256), bytes);
+}
+
+q8_status q8_q6k_gemv_packed(const void *packed, const float *x, float *y, int64_t M, int64_t K, int64_t N,
+                             q8_stream_t stream) {
+    return run_q6k_packed(packed, x, y, M, K, N, (cudaStream_t)stream);
 }
 
 q8_status q8_gemv_residual(const void *W, const float *x, const float *residual, float *y, int64_t M,

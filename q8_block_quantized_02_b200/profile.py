@@ -52,7 +52,8 @@ if ROOT not in sys.path:
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--op", choices=["gemv", "argmax", "swiglu", "q8q8", "q4k", "q6k", "moe", "readpeak", "decode"],
+    ap.add_argument("--op", choices=["gemv", "argmax", "swiglu", "q8q8", "q4k", "q6k", "q6kp", "moe", "readpeak",
+                             "decode"],
                     default="gemv",
                     help="q8_gemv, q8_gemv_argmax (logits not written), q8_gate_up_swiglu (M = rows of "
                          "the stacked gate|up matrix) or q8_quantize_act + q8q8_gemv (only q8q8_gemv is "
@@ -64,6 +65,8 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--copies", type=int, default=0, help="packed weight copies (0: cover 3x L2)")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--split", action="store_true",
+                    help="gemv / swiglu: the _split entry points (tensor cores where they serve)")
     ap.add_argument("--T", type=int, default=1, help="moe: tokens")
     ap.add_argument("--E", type=int, default=60, help="moe: routed experts")
     ap.add_argument("--H", type=int, default=2048, help="moe: hidden size")
@@ -87,7 +90,7 @@ def main(argv=None) -> int:
 
     M, K, N = args.M, args.K, args.N
     dev = torch.device("cuda", torch.cuda.current_device())
-    if args.op in ("q4k", "q6k"):
+    if args.op in ("q4k", "q6k", "q6kp"):
         return _kquant(args, q8, q8gen, np, torch, dev)
     g, x = q8gen.q8_matrix(args.seed, M, K, N)
     nbytes = q8.q8_packed_bytes(M, K)
@@ -120,11 +123,14 @@ def main(argv=None) -> int:
         p = packs[it[0] % copies]
         it[0] += 1
         if args.op == "gemv":
-            q8.q8_gemv(p, xf, y, M, K, N)
+            (q8.q8_gemv_split if args.split else q8.q8_gemv)(p, xf, y, M, K, N)
         elif args.op == "argmax":
             q8.q8_gemv_argmax(p, xf, None, M, K, N, best)
         elif args.op == "swiglu":
-            q8.q8_gate_up_swiglu(p, xf, y, M // 2, K, N)
+            if args.split:
+                q8.q8_gate_up_swiglu_split(p, xf, y, M // 2, K, N)
+            else:
+                q8.q8_gate_up_swiglu(p, xf, y, M // 2, K, N)
         else:
             q8.q8q8_gemv(p, xq, xd, y, M, K, N)
 
@@ -148,19 +154,27 @@ def main(argv=None) -> int:
 
 
 def _kquant(args, q8, q8gen, np, torch, dev) -> int:
-    """q8_q4k_gemv / q8_q6k_gemv on raw GGUF K-quant blocks (random fields);
-    bytes per call are the blocks' (144 or 210 per 256 weights)."""
+    """q8_q4k_gemv / q8_q6k_gemv on raw GGUF K-quant blocks (random fields), or
+    q8_q6k_gemv_packed (q6kp) on their packed units; bytes per call are the
+    blocks' (144 or 210 per 256 weights)."""
     M, K, N = args.M, args.K, args.N
     fmt = "q4_k" if args.op == "q4k" else "q6_k"
     blocks = q8gen.kquant_matrix(fmt, args.seed, M, K)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     copies = args.copies if args.copies > 0 else max(1, int(np.ceil(3 * l2 / blocks.size)))
     src = torch.from_numpy(blocks).to(dev)
-    ws = [src.clone() for _ in range(copies)]
+    if args.op == "q6kp":
+        ws = []
+        for _ in range(copies):
+            p = torch.empty(q8.q8_q6k_packed_bytes(M, K), dtype=torch.uint8, device=dev)
+            q8.q8_q6k_pack_weights(src, M, K, p)
+            ws.append(p)
+    else:
+        ws = [src.clone() for _ in range(copies)]
     del src
     x = torch.from_numpy(q8gen.activations(args.seed + 1, N, K)).to(dev)
     y = torch.empty((N, M), dtype=torch.float32, device=dev)
-    fn = q8.q8_q4k_gemv if fmt == "q4_k" else q8.q8_q6k_gemv
+    fn = {"q4k": q8.q8_q4k_gemv, "q6k": q8.q8_q6k_gemv, "q6kp": q8.q8_q6k_gemv_packed}[args.op]
     for i in range(args.warmup):
         fn(ws[i % copies], x, y, M, K, N)
     torch.cuda.synchronize()

@@ -124,6 +124,17 @@ def test_packed_bytes(lib):
     assert f(0, 32) == 0 and f(8, 0) == 0 and f(8, 48) == 0 and f(-8, 32) == 0
 
 
+def test_q6k_packed_bytes(lib):
+    f = lib.q8_q6k_packed_bytes
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    # one 6720-byte unit per (tile of 32 rows, 256-weight block)
+    assert f(32, 256) == 6720
+    assert f(33, 512) == 2 * 2 * 6720
+    assert f(152064, 3584) == 4752 * 14 * 6720
+    assert f(0, 256) == 0 and f(8, 300) == 0 and f(8, 0) == 0
+
+
 def test_status_strings(lib):
     f = lib.q8_status_string
     f.restype = ctypes.c_char_p
@@ -189,11 +200,16 @@ def test_host_validation_runs_before_any_device_work(lib):
     assert qq(n, n, n, n, 8, 32, 17, n) == 5
     bd = fn("q8q8_block_dots", P, P, P, I64, I64, I64, P)
     assert bd(n, n, n, 8, 20, 1, n) == 2
-    for name in ("q8_q4k_gemv", "q8_q6k_gemv"):
+    for name in ("q8_q4k_gemv", "q8_q6k_gemv", "q8_q6k_gemv_packed"):
         kq = fn(name, P, P, P, I64, I64, I64, P)
         assert kq(n, n, n, 8, 896, 1, n) == 2       # K % 256
         assert kq(n, n, n, 8, 512, 5, n) == 5       # N > 4
         assert kq(n, n, n, 8, 512, 1, n) == 1
+    for name in ("q8_q6k_pack_weights", "q8_q6k_unpack_weights"):
+        pk = fn(name, P, I64, I64, P, P)
+        assert pk(n, 8, 300, n, n) == 2             # K % 256
+        assert pk(n, 0, 256, n, n) == 2             # M <= 0
+        assert pk(n, 8, 256, n, n) == 1             # null pointers
     route = fn("q8_moe_route", P, I64, I64, I64, ctypes.c_int, P, P, P)
     assert route(n, 1, 4, 5, 0, n, n, n) == 2       # top_k > E
     assert route(n, 17, 60, 4, 0, n, n, n) == 5     # T > 16

@@ -100,3 +100,104 @@ def test_q4k_zero_weight_sub_blocks(N):
     y = run("q4_k", flat, x, M, K)
     y_ref, y_abs = oracle.kquant_gemv("q4_k", flat, x, M, K, threads=oracle.max_threads())
     assert_within(y, y_ref, TOL_REL * y_abs, f"q4_k zero-weight sub-blocks N={N}")
+
+
+# ---------------------------------------------------------------------------
+# Q6_K packed units (q8_q6k_pack_weights / q8_q6k_gemv_packed)
+# ---------------------------------------------------------------------------
+def pack_q6k_reference(blocks, M, K):
+    """The packed layout as include/q8.h states it, written with numpy: unit
+    (t, b) of 6720 bytes; row i of tile t at byte 208 i holds raw bytes 0..207
+    of block b of matrix row 32t + i, bytes 6656 + 2i, + 1 its d; rows past M
+    zero."""
+    SB = K // 256
+    T = -(-M // 32)
+    raw = np.zeros((T * 32, SB, 210), np.uint8)
+    raw[:M] = blocks.reshape(M, SB, 210)
+    raw = raw.reshape(T, 32, SB, 210).transpose(0, 2, 1, 3)  # [t][b][i][210]
+    out = np.zeros((T, SB, 6720), np.uint8)
+    out[:, :, :6656] = raw[:, :, :, :208].reshape(T, SB, 6656)
+    out[:, :, 6656:] = raw[:, :, :, 208:].reshape(T, SB, 64)
+    return out.reshape(-1)
+
+
+def pack_q6k(blocks, M, K):
+    t = torch()
+    raw = t.from_numpy(blocks.copy()).cuda()
+    packed = t.full((q8().q8_q6k_packed_bytes(M, K),), 0xA5, dtype=t.uint8, device="cuda")
+    q8().q8_q6k_pack_weights(raw, M, K, packed)
+    return packed
+
+
+def run_q6k_packed(packed, x, M, K):
+    t = torch()
+    N = x.shape[0]
+    y = t.full((N, M), float("nan"), dtype=t.float32, device="cuda")
+    q8().q8_q6k_gemv_packed(packed, dev(x), y, M, K, N)
+    return y.cpu().numpy()
+
+
+@pytest.mark.parametrize("M,K", [(1, 256), (45, 512), (100, 3584), (64, 18944)])
+def test_q6k_pack_layout_and_round_trip(M, K):
+    t = torch()
+    blocks = q8gen.kquant_matrix("q6_k", 91 + M, M, K)
+    packed = pack_q6k(blocks, M, K)
+    assert packed.numel() == -(-M // 32) * (K // 256) * 6720
+    assert np.array_equal(packed.cpu().numpy(), pack_q6k_reference(blocks, M, K))
+    raw = t.full((blocks.size,), 0x5A, dtype=t.uint8, device="cuda")
+    q8().q8_q6k_unpack_weights(packed, M, K, raw)
+    assert np.array_equal(raw.cpu().numpy(), blocks)
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 256, 1), (13, 512, 2), (1000, 3584, 4), (37, 2048, 3),
+                                   (3584, 18944, 1), (4096, 3584, 2), (33, 256, 1),
+                                   (4739, 2304, 1), (70, 4864, 2), (5000, 1024, 2),
+                                   # several tiles per CTA: the partial-sum buffers and
+                                   # their barriers go round more than once
+                                   (30000, 512, 1), (20000, 768, 2), (20000, 768, 3)])
+def test_q6k_packed_gemv_matches_oracle(M, K, N):
+    blocks = q8gen.kquant_matrix("q6_k", 5 * M + K + N, M, K)
+    x = q8gen.activations(M + 2 * K + N, N, K)
+    y = run_q6k_packed(pack_q6k(blocks, M, K), x, M, K)
+    y_ref, y_abs = oracle.kquant_gemv("q6_k", blocks, x, M, K, threads=oracle.max_threads())
+    assert_within(y, y_ref, TOL_REL * y_abs, f"q6_k packed M={M} K={K} N={N}")
+
+
+@pytest.mark.parametrize("M,K,N", [(30000, 512, 1), (20000, 768, 2)])
+def test_q4k_tile_many_tiles_per_cta(M, K, N):
+    blocks = q8gen.kquant_matrix("q4_k", 7 * M + K, M, K)
+    x = q8gen.activations(M + K + N, N, K)
+    y = run("q4_k", blocks, x, M, K)
+    y_ref, y_abs = oracle.kquant_gemv("q4_k", blocks, x, M, K, threads=oracle.max_threads())
+    assert_within(y, y_ref, TOL_REL * y_abs, f"q4_k M={M} K={K} N={N}")
+
+
+def test_q6k_packed_full_size_sampled_and_deterministic():
+    """152064 x 3584 at N = 1 and 2 from the packed units, sampled rows; two
+    runs bit-identical."""
+    M, K = 152064, 3584
+    blocks = q8gen.kquant_matrix("q6_k", 779, M, K)
+    packed = pack_q6k(blocks, M, K)
+    rows = np.unique(np.concatenate([np.arange(4), np.arange(M - 4, M),
+                                     np.random.default_rng(1).integers(0, M, 200)]))
+    sub = blocks.reshape(M, (K // 256) * 210)[rows].reshape(-1)
+    for N in (1, 2):
+        x = q8gen.activations(780 + N, N, K)
+        y = run_q6k_packed(packed, x, M, K)
+        assert np.array_equal(y, run_q6k_packed(packed, x, M, K))
+        y_ref, y_abs = oracle.kquant_gemv("q6_k", sub, x, len(rows), K, threads=oracle.max_threads())
+        assert_within(y[:, rows], y_ref, TOL_REL * y_abs, f"q6_k packed full size N={N}")
+
+
+def test_q6k_packed_rejections():
+    t = torch()
+    M, K = 64, 512
+    packed = t.zeros((q8().q8_q6k_packed_bytes(M, K),), dtype=t.uint8, device="cuda")
+    y = t.empty((5, M), dtype=t.float32, device="cuda")
+    assert q8().q8_q6k_packed_bytes(M, 300) == 0
+    with pytest.raises(q8().Q8Error) as e:
+        q8().q8_q6k_gemv_packed(packed, dev(np.zeros((5, K), np.float32)), y, M, K, 5)  # N > 4
+    assert e.value.status == 5
+    with pytest.raises(q8().Q8Error) as e:
+        q8().q8_q6k_gemv_packed(packed[1:], dev(np.zeros((1, K), np.float32)), y, M, K, 1)  # unaligned
+    assert e.value.status == 3
