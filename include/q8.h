@@ -207,8 +207,8 @@ static inline float q8_argmax_value(uint64_t key) {
  * blocks).  W: [M][K/256] blocks, rows contiguous, unpacked.  x: [N][K] fp32,
  * 16-byte aligned.  y: [N][M] fp32.  K % 256 == 0; 1 <= N <= 4.  Each output
  * is within 1e-5 * sum_k |w x| of the exact value (every weight formed with
- * at most one fp32 rounding).  CUDA cores: Q4_K at N <= 2 in tiles of 32 rows
- * fed by TMA boxes, otherwise one warp per row.
+ * at most one fp32 rounding).  CUDA cores: Q4_K in tiles of 32 rows fed by
+ * TMA boxes (activation rows two per launch), Q6_K one warp per row.
  * Q4_K, 144-byte blocks, W 16-byte aligned: d (binary16) | dmin (binary16) |
  *   scales[12] | qs[128].  Sub-block j (weights 32j..32j+31) has a 6-bit
  *   scale sc and min m: j < 4: sc = scales[j] & 63, m = scales[j+4] & 63;

@@ -128,32 +128,6 @@ struct FmArgs {
     const float *res;  // GEMV: [N][M_out] added to the outputs (q8_gemv_residual; may be y), or null
 };
 
-__device__ __forceinline__ void tmem_ld4_async(uint32_t taddr, uint32_t *v) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
-                 : "r"(taddr)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_ld1_async(uint32_t taddr, uint32_t *v) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v[0]) : "r"(taddr) : "memory");
-}
-__device__ __forceinline__ void tmem_ld2_async(uint32_t taddr, uint32_t *v) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];"
-                 : "=r"(v[0]), "=r"(v[1])
-                 : "r"(taddr)
-                 : "memory");
-}
-// Waits for every earlier tcgen05.ld of the thread; names 8 of the loaded
-// registers so that no use of them is scheduled before it (called once per
-// 8 registers: the later calls return at once).
-__device__ __forceinline__ void tmem_wait_ld8(uint32_t *v) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]),
-                   "+r"(v[7])
-                 :
-                 : "memory");
-}
-
 // The low byte of four words, in order, as one word.
 __device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);

@@ -11,13 +11,13 @@
 //   Q6_K, 210 B: ql[128] | qh[64] | scales[16] (int8, per 16 weights) | d.
 //   w = d*scale*(q - 32), q = 4 low bits from ql, 2 high bits from qh.
 //
-// The first kernel (every Q6_K product, and Q4_K at N = 3, 4): one warp per
-// output row (grid-stride); lane l takes the 32-weight chunks
-// l, l + 32, ... of the row: it decodes its chunk's scale (and min) once,
-// forms each weight with one fp32 FMA (Q4_K: d*sc*q - dmin*m; Q6_K:
-// d*scale*(q-32), exact), and multiplies it into every activation row.
-// Lanes' partial sums meet in a fixed shuffle tree, so results are
-// bit-identical from run to run.
+// Q6_K on raw blocks (q8_q6k_gemv): one warp per output row (grid-stride);
+// lane l takes the 32-weight chunks l, l + 32, ... of the row, decodes the
+// chunk's two scales once, forms each weight d*scale*(q-32) exactly in fp32
+// and multiplies it into every activation row.  Lanes' partial sums meet in a
+// fixed shuffle tree, so results are bit-identical from run to run.  Raw
+// blocks start on 2-byte boundaries, so this kernel reads bytes; the packed
+// units below serve the tile kernel.
 #pragma once
 
 #include "q8_device.cuh"
@@ -25,17 +25,6 @@
 namespace q8 {
 
 constexpr int kKqThreads = 256;
-
-// Sub-block j's 6-bit scale and min from the 12 packed bytes of a Q4_K block.
-__device__ __forceinline__ void q4k_scale_min(const uint8_t *s, int j, int &sc, int &m) {
-    if (j < 4) {
-        sc = s[j] & 63;
-        m = s[j + 4] & 63;
-    } else {
-        sc = (s[j + 4] & 15) | ((s[j - 4] >> 6) << 4);
-        m = (s[j + 4] >> 4) | ((s[j] >> 6) << 4);
-    }
-}
 
 // acc[n] += sum over 8 weights w[0..7] of w * x[n][k0 .. k0 + 7]
 template <int NMAX>
@@ -60,14 +49,13 @@ __device__ __forceinline__ void kq_dot8(const float (&w)[8], const float *__rest
     }
 }
 
-// FMT 4: Q4_K; FMT 6: Q6_K.
-template <int NMAX, int FMT>
-__global__ void __launch_bounds__(kKqThreads) kquant_gemv_kernel(const uint8_t *__restrict__ W,
-                                                                 const float *__restrict__ x,
-                                                                 float *__restrict__ y, int M, int K, int N) {
+template <int NMAX>
+__global__ void __launch_bounds__(kKqThreads) q6k_row_kernel(const uint8_t *__restrict__ W,
+                                                             const float *__restrict__ x,
+                                                             float *__restrict__ y, int M, int K, int N) {
     pdl_wait();
     pdl_launch_dependents();
-    constexpr int BYTES = FMT == 4 ? 144 : 210;
+    constexpr int BYTES = 210;
     const int lane = threadIdx.x & 31;
     const int SB = K / 256, chunks = K / 32;
     const int warps = (int)(gridDim.x * (kKqThreads / 32));
@@ -79,50 +67,24 @@ __global__ void __launch_bounds__(kKqThreads) kquant_gemv_kernel(const uint8_t *
             const uint8_t *blk = W + ((size_t)row * SB + (c >> 3)) * BYTES;
             const int cc = c & 7;
             const int64_t k0 = (int64_t)c * 32;
-            if (FMT == 4) {
-                const uint32_t dw = *reinterpret_cast<const uint32_t *>(blk);
-                const float d = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu)));
-                const float dmin = __half2float(__ushort_as_half((unsigned short)(dw >> 16)));
-                int sc, m;
-                q4k_scale_min(blk + 4, cc, sc, m);
-                const float a = d * (float)sc, b = dmin * (float)m;  // both exact in fp32
-                const uint4 *qs = reinterpret_cast<const uint4 *>(blk + 16 + 32 * (cc >> 1));
-                const int shift = 4 * (cc & 1);
+            const int hh = cc >> 2, c4 = cc & 3;
+            const uint8_t *ql = blk + 64 * hh + 32 * (c4 & 1);
+            const uint8_t *qh = blk + 128 + 32 * hh;
+            const int8_t *scl = reinterpret_cast<const int8_t *>(blk + 192 + 8 * hh + 2 * c4);
+            const float d = __half2float(__ushort_as_half(
+                (unsigned short)(blk[208] | ((unsigned)blk[209] << 8))));
+            const float a0 = d * (float)scl[0], a1 = d * (float)scl[1];  // exact in fp32
+            const int lshift = 4 * (c4 >> 1), hshift = 2 * c4;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint4 v = qs[h];
-                    const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+            for (int p = 0; p < 4; ++p) {
+                float w[8];
 #pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        float w[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const uint32_t byte = (words[2 * p + (i >> 2)] >> (8 * (i & 3))) & 0xFFu;
-                            w[i] = fmaf(a, (float)((byte >> shift) & 15u), -b);
-                        }
-                        kq_dot8<NMAX>(w, x, K, N, k0 + 16 * h + 8 * p, acc);
-                    }
+                for (int i = 0; i < 8; ++i) {
+                    const int l = 8 * p + i;
+                    const int q = (int)(((ql[l] >> lshift) & 15) | (((qh[l] >> hshift) & 3) << 4)) - 32;
+                    w[i] = (l < 16 ? a0 : a1) * (float)q;  // exact: 11 x 8 x 6 significant bits
                 }
-            } else {
-                const int hh = cc >> 2, c4 = cc & 3;
-                const uint8_t *ql = blk + 64 * hh + 32 * (c4 & 1);
-                const uint8_t *qh = blk + 128 + 32 * hh;
-                const int8_t *scl = reinterpret_cast<const int8_t *>(blk + 192 + 8 * hh + 2 * c4);
-                const float d = __half2float(__ushort_as_half(
-                    (unsigned short)(blk[208] | ((unsigned)blk[209] << 8))));
-                const float a0 = d * (float)scl[0], a1 = d * (float)scl[1];  // exact in fp32
-                const int lshift = 4 * (c4 >> 1), hshift = 2 * c4;
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    float w[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int l = 8 * p + i;
-                        const int q = (int)(((ql[l] >> lshift) & 15) | (((qh[l] >> hshift) & 3) << 4)) - 32;
-                        w[i] = (l < 16 ? a0 : a1) * (float)q;  // exact: 11 x 8 x 6 significant bits
-                    }
-                    kq_dot8<NMAX>(w, x, K, N, k0 + 8 * p, acc);
-                }
+                kq_dot8<NMAX>(w, x, K, N, k0 + 8 * p, acc);
             }
         }
 #pragma unroll
@@ -245,20 +207,16 @@ __device__ __forceinline__ void q4_weights(const uint4 v, uint64_t a0, uint64_t 
     }
 }
 
-// The 6-bit scale and min of sub-block j from the 12 scale bytes held in the
-// words s1 (bytes 0-3), s2 (4-7), s3 (8-11), as small exact floats.
-__device__ __forceinline__ void q4_sc_m(uint32_t s1, uint32_t s2, uint32_t s3, int j, float &sc, float &m) {
-    uint32_t a, b;
-    if (j < 4) {
-        a = (s1 >> (8 * j)) & 63u;
-        b = (s2 >> (8 * j)) & 63u;
-    } else {
-        const int k = 8 * (j - 4);
-        a = ((s3 >> k) & 15u) | (((s1 >> k) >> 6 & 3u) << 4);
-        b = ((s3 >> k) >> 4 & 15u) | (((s2 >> k) >> 6 & 3u) << 4);
-    }
-    sc = __uint_as_float(0x4B000000u | a) - 8388608.0f;
-    m = __uint_as_float(0x4B000000u | b) - 8388608.0f;
+// Sub-block j's 6-bit scale (bits 0..5) and min (bits 16..21) from the 12
+// scale bytes held in s1 (bytes 0-3), s2 (4-7), s3 (8-11), without a branch
+// on j: j < 4 takes the low 6 bits of bytes j and j + 4; j >= 4 takes the
+// nibbles of byte j + 4 and the top 2 bits of bytes j - 4 and j.
+__device__ __forceinline__ uint32_t q4_sc_m_packed(uint32_t s1, uint32_t s2, uint32_t s3, int j) {
+    const uint32_t sel = 0x4440u | (uint32_t)(j & 3);  // byte j % 4 into byte 0, zeros above
+    const uint32_t c1 = __byte_perm(s1, 0u, sel), c2 = __byte_perm(s2, 0u, sel), c3 = __byte_perm(s3, 0u, sel);
+    const uint32_t sc = j < 4 ? (c1 & 63u) : ((c3 & 15u) | ((c1 >> 2) & 0x30u));
+    const uint32_t m = j < 4 ? (c2 & 63u) : ((c3 >> 4) | ((c2 >> 2) & 0x30u));
+    return sc | (m << 16);
 }
 
 // q - 32 of the 16 Q6_K values of one run as fp32 pairs: 4 low bits per byte
@@ -410,13 +368,19 @@ __global__ void __launch_bounds__(kKqTileThreads, MINB)
                         const uint4 qv = *reinterpret_cast<const uint4 *>(blk + 16 + 16 * u);  // piece u
                         const float d = __half2float(__ushort_as_half((unsigned short)(hd.x & 0xFFFFu)));
                         const float dmin = __half2float(__ushort_as_half((unsigned short)(hd.x >> 16)));
-                        const int t = u >> 1;
-                        float sc0, m0, sc1, m1;
-                        q4_sc_m(hd.y, hd.z, hd.w, 2 * t, sc0, m0);
-                        q4_sc_m(hd.y, hd.z, hd.w, 2 * t + 1, sc1, m1);
-                        // d*sc and dmin*m are exact in fp32 (11 x 6 significant bits)
-                        const uint32_t a0 = __float_as_uint(d * sc0), b0 = __float_as_uint(-(dmin * m0));
-                        const uint32_t a1 = __float_as_uint(d * sc1), b1 = __float_as_uint(-(dmin * m1));
+                        // lane u decodes sub-block u's scale and min; this lane's
+                        // sub-blocks 2t, 2t + 1 come from lanes 2t, 2t + 1 of its row
+                        const uint32_t scm = q4_sc_m_packed(hd.y, hd.z, hd.w, u);
+                        const int t = u >> 1, base = lane & ~7;
+                        const uint32_t p0 = __shfl_sync(0xffffffffu, scm, base + 2 * t);
+                        const uint32_t p1 = __shfl_sync(0xffffffffu, scm, base + 2 * t + 1);
+                        // d*sc and dmin*m are exact in fp32 (11 x 6 significant bits):
+                        // d * (2^23 + sc) - d * 2^23 in one fma
+                        const float d23 = d * 8388608.0f, dm23 = dmin * 8388608.0f;
+                        const uint32_t a0 = __float_as_uint(fmaf(d, __uint_as_float(0x4B000000u | (p0 & 63u)), -d23));
+                        const uint32_t b0 = __float_as_uint(fmaf(-dmin, __uint_as_float(0x4B000000u | (p0 >> 16)), dm23));
+                        const uint32_t a1 = __float_as_uint(fmaf(d, __uint_as_float(0x4B000000u | (p1 & 63u)), -d23));
+                        const uint32_t b1 = __float_as_uint(fmaf(-dmin, __uint_as_float(0x4B000000u | (p1 >> 16)), dm23));
                         uint64_t wl[8], wh[8];
                         q4_weights(qv, pack_u32x2(a0, a0), pack_u32x2(b0, b0), pack_u32x2(a1, a1), pack_u32x2(b1, b1),
                                    wl, wh);

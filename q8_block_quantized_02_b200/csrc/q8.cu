@@ -410,7 +410,7 @@ static q8_status run_tile(const void *W, const void *x, const uint16_t *xd, floa
 #define Q8_MMA_MIN_N 5
 #endif
 constexpr int64_t kMmaMinN = Q8_MMA_MIN_N;  // smallest N sent to the tcgen05 kernel
-constexpr int kMmaMaxStages = 3;
+constexpr int kMmaMaxStages = 2;  // 78 KB stages: 32 columns (4 KB per group) keep HBM bursts long
 
 static cudaError_t setup_mma_kernel(int max_smem) {
     const void *k = reinterpret_cast<const void *>(&q8q8_mma_kernel);
@@ -844,8 +844,8 @@ static q8_status kquant_check(const void *W, const float *x, float *y, int64_t M
 }
 
 template <int FMT>
-// K-quant GEMV on raw blocks: argument checks, then the tile kernel (Q4_K,
-// N <= 2) or one warp per row.
+// K-quant GEMV on raw blocks: argument checks, then the tile kernel (Q4_K)
+// or one warp per row (Q6_K on raw blocks).
 static q8_status run_kquant(const void *W, const float *x, float *y, int64_t M, int64_t K, int64_t N,
                             cudaStream_t stream, const char *name) {
     Q8_CHECK(kquant_check(W, x, y, M, K, N, FMT == 4));  // Q4_K blocks are read as aligned words / TMA boxes
@@ -853,22 +853,30 @@ static q8_status run_kquant(const void *W, const float *x, float *y, int64_t M, 
     Q8_CHECK(device_info(&dev));
     const int nm = (int)N;
     const uint8_t *w8 = static_cast<const uint8_t *>(W);
-    if (FMT == 4 && N <= 2) {
-        // raw rows of 144 * SB bytes: boxes of {one 144-byte block, 32 rows}
+    if constexpr (FMT == 4) {
+        // raw rows of 144 * SB bytes: boxes of {one 144-byte block, 32 rows};
+        // activation rows two per launch
         const int64_t SB = K / 256;
         CUtensorMap map;
         const q8_status ms =
             make_map_3d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, 144, SB, M, 144, 144 * SB, 144, 1, kKqRows, true);
         if (ms != Q8_OK) return ms;
-        return N == 1 ? launch_kq_tile<4, 1, 3, 2>(map, w8, x, y, M, K, nm, dev->sms, stream, name)
-                      : launch_kq_tile<4, 2, 4, 1>(map, w8, x, y, M, K, nm, dev->sms, stream, name);
-    }
-    const int64_t warps = std::min<int64_t>(M, (int64_t)dev->sms * 64);
-    const unsigned grid = (unsigned)ceil_div(warps, kKqThreads / 32);
-    switch (nmax_for(N)) {
-        case 1: return launch_pdl(kquant_gemv_kernel<1, FMT>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
-        case 2: return launch_pdl(kquant_gemv_kernel<2, FMT>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
-        default: return launch_pdl(kquant_gemv_kernel<4, FMT>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
+        for (int64_t n0 = 0; n0 < N; n0 += 2) {
+            const int nn = (int)std::min<int64_t>(2, N - n0);
+            const q8_status st =
+                nn == 1 ? launch_kq_tile<4, 1, 3, 2>(map, w8, x + n0 * K, y + n0 * M, M, K, 1, dev->sms, stream, name)
+                        : launch_kq_tile<4, 2, 4, 1>(map, w8, x + n0 * K, y + n0 * M, M, K, 2, dev->sms, stream, name);
+            if (st != Q8_OK) return st;
+        }
+        return Q8_OK;
+    } else {
+        const int64_t warps = std::min<int64_t>(M, (int64_t)dev->sms * 64);
+        const unsigned grid = (unsigned)ceil_div(warps, kKqThreads / 32);
+        switch (nmax_for(N)) {
+            case 1: return launch_pdl(q6k_row_kernel<1>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
+            case 2: return launch_pdl(q6k_row_kernel<2>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
+            default: return launch_pdl(q6k_row_kernel<4>, dim3(grid), dim3(kKqThreads), 0, stream, name, w8, x, y, (int)M, (int)K, nm);
+        }
     }
 }
 

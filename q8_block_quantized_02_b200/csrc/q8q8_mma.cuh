@@ -20,11 +20,12 @@
 //     Stored bytes are q + 128, so A is read as unsigned 8-bit;
 //   * B = activations, N = 16 rows (zero padded past N) x 32 bytes, loaded
 //     as [column][row][16 B] (core matrices of 8 rows), read as signed 8-bit;
-//   * D = 128 lanes x 16 int32 columns of tensor memory per block: block j
-//     of a stage lands at column 16 j, and each epilogue warp takes a half
-//     stage (4 blocks, 64 columns) with one tcgen05.ld, so the load latency is
-//     paid once per 4 blocks; the MMA fills one half while the epilogue reads
-//     the other.
+//   * D = 128 lanes x 16 int32 columns of tensor memory per block.  A half
+//     stage (4 blocks, 64 columns) fills the next slot of a ring of 8 such
+//     slots (all 512 columns), so the MMAs run up to two stages ahead of the
+//     epilogue and their latency stays off its path; each epilogue warp
+//     loads its columns of a half before one wait, paying the load latency
+//     once per 4 blocks.
 // Because A holds q + 128, the tensor cores return dot + 128 * sum_i xq[n][i];
 // the epilogue removes that term exactly.  Its int -> float conversion adds
 // the correction to 0x4B400000 (the bits of 1.5 * 2^23) and subtracts
@@ -50,21 +51,23 @@ namespace q8 {
 
 constexpr int kMmaTileGroups = 16;                 // 128 output rows per tile
 constexpr int kMmaN = 16;                          // MMA N: activation columns (padded)
-constexpr int kMmaCS = 16;                         // 16-byte columns per stage
+constexpr int kMmaCS = 32;                         // 16-byte columns per stage: 4 KB of each group
 constexpr int kMmaSB = kMmaCS / 2;                 // blocks per stage
 constexpr int kMmaHalfBlocks = 4;                  // blocks per TMEM half (one ld each)
 constexpr int kMmaHalves = kMmaSB / kMmaHalfBlocks;   // TMEM halves per stage
-constexpr uint32_t kMmaTmemCols = kMmaSB * kMmaN;     // 128 columns: block j at column 16 j
+constexpr int kMmaTSlots = 8;                         // TMEM ring of halves (two stages)
+constexpr uint32_t kMmaSlotCols = kMmaHalfBlocks * kMmaN;      // 64 columns a half
+constexpr uint32_t kMmaTmemCols = kMmaTSlots * kMmaSlotCols;  // 512 columns
 constexpr int kMmaEpiGroups = 2;                   // epilogue warp groups, split over n
 constexpr int kMmaNPG = kMmaN / kMmaEpiGroups;     // activation columns per group
 constexpr int kMmaEpiThreads = kMmaEpiGroups * 128;
 constexpr int kMmaThreads = 64 + kMmaEpiThreads;   // producer, MMA, epilogue
 constexpr int kMmaMaxSplit = 8;
 
-constexpr uint32_t kMmaQBytes = kMmaCS * kMmaTileGroups * kColBytes;  // 32 KB
-constexpr uint32_t kMmaDBytes = kMmaSB * kMmaTileGroups * 16;         // 2 KB
-constexpr uint32_t kMmaXBytes = kMmaCS * kMmaN * 16;                  // 4 KB
-constexpr uint32_t kMmaTabBytes = kMmaSB * kMmaN * 8;                 // 1 KB
+constexpr uint32_t kMmaQBytes = kMmaCS * kMmaTileGroups * kColBytes;  // 64 KB
+constexpr uint32_t kMmaDBytes = kMmaSB * kMmaTileGroups * 16;         // 4 KB
+constexpr uint32_t kMmaXBytes = kMmaCS * kMmaN * 16;                  // 8 KB
+constexpr uint32_t kMmaTabBytes = kMmaSB * kMmaN * 8;                 // 2 KB
 constexpr uint32_t kMmaDOff = kMmaQBytes;
 constexpr uint32_t kMmaXOff = kMmaDOff + kMmaDBytes;
 constexpr uint32_t kMmaTabOff = kMmaXOff + kMmaXBytes;
@@ -74,7 +77,7 @@ constexpr uint32_t kMmaRedBytes = kMmaN * 128 * 4;                    // one til
 
 // Shared-memory carve-up (host and device): stages, barriers, partials, misc.
 __host__ __device__ constexpr uint32_t mma_bar_off(int stages) { return stages * kMmaStageBytes; }
-__host__ __device__ constexpr uint32_t mma_nbars(int stages) { return 2 * stages + 2 * kMmaHalves + 3; }
+__host__ __device__ constexpr uint32_t mma_nbars(int stages) { return 2 * stages + 2 * kMmaTSlots + 3; }
 __host__ __device__ constexpr uint32_t mma_red_off(int stages) {
     return (mma_bar_off(stages) + 8 * mma_nbars(stages) + 127) / 128 * 128;
 }
@@ -144,9 +147,9 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
                  : "memory");
 }
 
-// 8 columns of 32 lanes, without waiting: the registers are undefined until
-// tmem_wait_ld32 below, which names them as operands so that no use of them
-// is scheduled before the wait.
+// Column loads of 32 lanes without waiting: the registers are undefined until
+// tmem_wait_ld8, which names them as operands so that no use of them is
+// scheduled before the wait.
 __device__ __forceinline__ void tmem_ld8_async(uint32_t taddr, uint32_t *v) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                  : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
@@ -154,16 +157,32 @@ __device__ __forceinline__ void tmem_ld8_async(uint32_t taddr, uint32_t *v) {
                  : "r"(taddr)
                  : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld32(uint32_t (&v)[32]) {
+__device__ __forceinline__ void tmem_ld4_async(uint32_t taddr, uint32_t *v) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                 : "r"(taddr)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld1_async(uint32_t taddr, uint32_t *v) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v[0]) : "r"(taddr) : "memory");
+}
+__device__ __forceinline__ void tmem_ld2_async(uint32_t taddr, uint32_t *v) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];"
+                 : "=r"(v[0]), "=r"(v[1])
+                 : "r"(taddr)
+                 : "memory");
+}
+// Waits for every earlier tcgen05.ld of the thread; names 8 of the loaded
+// registers so that no use of them is scheduled before it (called once per
+// 8 registers: the later calls return at once).
+__device__ __forceinline__ void tmem_wait_ld8(uint32_t *v) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]),
-                   "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]),
-                   "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]),
-                   "+r"(v[21]), "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]),
-                   "+r"(v[28]), "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+                   "+r"(v[7])
                  :
                  : "memory");
 }
+
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -239,8 +258,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     const uint32_t full0 = smem_u32(smem + mma_bar_off(a.stages));
     const uint32_t empty0 = full0 + 8 * a.stages;
     const uint32_t tfull0 = empty0 + 8 * a.stages;
-    const uint32_t tempty0 = tfull0 + 8 * kMmaHalves;
-    const uint32_t done_bar = tempty0 + 8 * kMmaHalves;
+    const uint32_t tempty0 = tfull0 + 8 * kMmaTSlots;
+    const uint32_t done_bar = tempty0 + 8 * kMmaTSlots;
     const uint32_t redfull = done_bar + 8, redfree = redfull + 8;
     float *red = reinterpret_cast<float *>(smem + mma_red_off(a.stages));
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + mma_misc_off(a.stages, S > 1));
@@ -274,7 +293,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1 + kMmaEpiThreads / 32);  // MMA commit + epilogue warps
         }
-        for (int h = 0; h < kMmaHalves; ++h) {
+        for (int h = 0; h < kMmaTSlots; ++h) {
             mbar_init(tfull0 + 8 * h, 1);
             mbar_init(tempty0 + 8 * h, kMmaEpiThreads / 32);
         }
@@ -346,9 +365,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         // ------------------------------ MMA issuer ----------------------------
         pdl_wait_and_trigger();  // its inputs arrive after the producer's wait anyway
         if (lane == 0) {
-            // Block j of every stage goes to TMEM columns 16 j; the two halves
-            // (blocks 0-3, 4-7) are each handed to the epilogue by one commit.
+            // Half h of each stage (blocks 4h .. 4h + 3) goes to the next slot
+            // of a ring of kMmaTSlots TMEM slots of 64 columns (block jj of
+            // the half at column 16 jj), handed to the epilogue by one commit;
+            // the MMAs run up to four stages ahead of the epilogue's reads.
             bool ok = true;
+            int ts = 0, tph = 0;  // TMEM slot and its phase, carried along
             int slot = 0, phase = 0, ks = 0;  // ring position and k step of iteration `it`
             for (int it = 0; it < total && ok;
                  ++it, ks = ks + 1 == ksteps ? 0 : ks + 1, slot = slot + 1 == a.stages ? 0 : slot + 1,
@@ -358,8 +380,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                 const int nb = min(kMmaSB, nblk - ks * kMmaSB);
                 const uint32_t st = smem_u32(smem + (size_t)slot * kMmaStageBytes);
                 for (int h = 0; h < kMmaHalves; ++h) {
-                    // the epilogue has read this half of the previous stage
-                    if (!mbar_wait(tempty0 + 8 * h, (it & 1) ^ 1, abort_flag)) {
+                    // the epilogue has read this slot's previous half
+                    if (!mbar_wait(tempty0 + 8 * ts, tph ^ 1, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -369,11 +391,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                         const uint64_t ad = mma_smem_desc(st + j * 2 * kColBytes, kColBytes, kMmaCS * kColBytes);
                         // activations [column][16 rows][16 B]: columns 256 B apart, 8-row halves 128 B
                         const uint64_t bd = mma_smem_desc(st + kMmaXOff + j * 2 * (kMmaN * 16), kMmaN * 16, 8 * 16);
-                        mma_i8(tmem + j * kMmaN, ad, bd, kMmaIdesc);
+                        mma_i8(tmem + ts * kMmaSlotCols + (j - h * kMmaHalfBlocks) * kMmaN, ad, bd, kMmaIdesc);
                     }
                     // past the end of K the half holds no new block: the commit
                     // still arrives, once the earlier MMAs are done
-                    mma_commit(tfull0 + 8 * h);
+                    mma_commit(tfull0 + 8 * ts);
+                    if (++ts == kMmaTSlots) { ts = 0; tph ^= 1; }
                 }
                 if (ok) mma_commit(empty0 + 8 * slot);
             }
@@ -436,6 +459,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
             }
         };
         int it = 0, slot = 0, phase = 0;  // ring position of iteration `it`, carried along
+        int ts = 0, tph = 0;              // TMEM slot of the next half and its phase
         for (int tl = 0; tl < n_tiles; ++tl) {
 #pragma unroll
             for (int p = 0; p < kMmaNPG / 2; ++p) acc2[p] = 0ull;
@@ -459,17 +483,24 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                 for (int h = 0; h < kMmaHalves && ok; ++h) {
                     const int j0 = h * kMmaHalfBlocks;
                     uint32_t v[kMmaHalfBlocks * kMmaNPG];
-                    const bool okh = mbar_wait_warp(tfull0 + 8 * h, it & 1, abort_flag);
+                    const bool okh = mbar_wait_warp(tfull0 + 8 * ts, tph, abort_flag);
                     if (okh && j0 < nb) {
                         tc_fence_after();
 #pragma unroll
-                        for (int jj = 0; jj < kMmaHalfBlocks; ++jj)
-                            tmem_ld8_async(taddr + (j0 + jj) * kMmaN, v + jj * kMmaNPG);
-                        tmem_wait_ld32(v);
+                        for (int jj = 0; jj < kMmaHalfBlocks; ++jj) {
+                            const uint32_t ta = taddr + ts * kMmaSlotCols + jj * kMmaN;
+                            if constexpr (kMmaNPG == 8)
+                                tmem_ld8_async(ta, v + jj * kMmaNPG);
+                            else
+                                tmem_ld4_async(ta, v + jj * kMmaNPG);
+                        }
+#pragma unroll
+                        for (int i = 0; i < kMmaHalfBlocks * kMmaNPG; i += 8) tmem_wait_ld8(v + i);
                         tc_fence_before();
                     }
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(tempty0 + 8 * h);
+                    if (lane == 0) mbar_arrive(tempty0 + 8 * ts);
+                    if (++ts == kMmaTSlots) { ts = 0; tph ^= 1; }
                     if (!okh) break;
                     // a full stage takes the branch-free path, so the four
                     // blocks' loads and arithmetic can interleave
