@@ -105,8 +105,9 @@ __global__ void __launch_bounds__(kKqThreads) q6k_row_kernel(const uint8_t *__re
 // The kernel above re-reads x for every row, and holds one row's loads at a
 // time.  Here a CTA of 8 warps takes tiles of kKqRows = 32 output rows; within
 // a tile, warp w takes super-blocks b = w', w' + 8, ... (w' = w rotated by
-// tile * SB, so that over a CTA's tiles every warp gets the same share when
-// SB is not a multiple of 8).  A warp's (tile, block) steps stream through its
+// i * SB for the CTA's i-th tile, so that over a few consecutive tiles every
+// warp gets the same share when SB is not a multiple of 8; rotating by the
+// global tile index would not, since a CTA's tiles are a grid apart).  A warp's (tile, block) steps stream through its
 // own ring of shared-memory stages, each holding one block of the tile's 32
 // rows and filled by one copy that lane 0 issues on the stage's mbarrier:
 //   * Q4_K: the raw rows are 144 * SB bytes, so a 3-D TMA box {144 B, 1 block,
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kKqThreads) q6k_row_kernel(const uint8_t *__re
 //   * Q4_K piece u = 2t + h: weights 64t + 16h + i (low nibbles, sub-block 2t)
 //     and 64t + 32 + 16h + i (high nibbles, sub-block 2t + 1), i < 16.  Each
 //     weight is fma(d*sc, q, -dmin*m) (d*sc and dmin*m exact in fp32), one
-//     rounding relative to itself, as in the kernel above: factoring the
+//     rounding relative to itself: factoring the
 //     sub-block's terms out of the sum would be cheaper, but its rounding
 //     would scale with d*sc*sum q x and dmin*m*sum x, not with sum |w x|, and
 //     the two cancel when the weights are near zero.
@@ -140,13 +141,15 @@ __global__ void __launch_bounds__(kKqThreads) q6k_row_kernel(const uint8_t *__re
 // mantissa bits of 2^23 by a byte permute it gives 2^23 + q exactly, and one
 // paired subtract removes the bias.  Dots use packed f32x2 FMAs.
 // Row sums: the 8 lanes of a row by a shuffle tree, then the 8 warps'
-// partials in warp order by one reducer warp per tile (warp tile % 8), so
-// results are bit-identical from run to run.  The partials go through two
-// shared buffers (tile parity) under named barriers: a warp arrives on the
-// tile's "full" barrier and moves on; only the reducer waits there.  Before
-// writing tile t's partials a warp waits on the buffer's "free" barrier, on
-// which the reducer of tile t - 2 arrives once it has read them.  So no
-// computing warp waits for a slower one, except across two tiles.
+// partials in warp order by one reducer warp per tile (warp i % 8 for the
+// CTA's i-th tile), so results are bit-identical from run to run (the
+// rotation depends on the grid, so they may differ between GPUs with
+// different SM counts).  The partials go through kKqRedBufs shared buffers
+// (tile i uses buffer i % 4) under named barriers: a warp arrives on the
+// buffer's "full" barrier and moves on; only the reducer waits there.  Before
+// writing tile i's partials a warp waits on the buffer's "free" barrier, on
+// which the reducer of tile i - 4 arrives once it has read them.  So no
+// computing warp waits for a slower one, except across four tiles.
 constexpr int kKqWarps = 8;
 constexpr int kKqTileThreads = kKqWarps * 32;
 constexpr int kKqRows = 32;                      // rows per tile (8 per lane)
@@ -154,6 +157,7 @@ constexpr int kQ4StageBytes = kKqRows * 144;     // 4608
 constexpr int kQ6RowBytes = 208;                 // ql | qh | scales of one row
 constexpr int kQ6UnitBytes = kKqRows * kQ6RowBytes + kKqRows * 2;  // 6720
 constexpr int kQ6DOff = kKqRows * kQ6RowBytes;   // 6656
+constexpr int kKqRedBufs = 4;                    // partial-sum buffers (tiles in flight)
 
 template <int FMT>
 __host__ __device__ constexpr int kq_stage_bytes() { return FMT == 4 ? kQ4StageBytes : kQ6UnitBytes; }
@@ -161,13 +165,13 @@ __host__ __device__ constexpr int kq_stage_bytes() { return FMT == 4 ? kQ4StageB
 template <int FMT, int NMAX, int STAGES>
 __host__ __device__ constexpr int kq_red_off() { return kKqWarps * STAGES * kq_stage_bytes<FMT>(); }
 template <int FMT, int NMAX, int STAGES>
-__host__ __device__ constexpr int kq_bar_off() { return kq_red_off<FMT, NMAX, STAGES>() + 2 * kKqWarps * NMAX * kKqRows * 4; }
+__host__ __device__ constexpr int kq_bar_off() { return kq_red_off<FMT, NMAX, STAGES>() + kKqRedBufs * kKqWarps * NMAX * kKqRows * 4; }
 template <int FMT, int NMAX, int STAGES>
 __host__ __device__ constexpr int kq_smem_bytes() { return kq_bar_off<FMT, NMAX, STAGES>() + kKqWarps * STAGES * 8 + 16; }
 
 // Named barriers of the partial-sum exchange (0 is __syncthreads').
-constexpr int kKqBarFull = 1;  // + tile parity
-constexpr int kKqBarFree = 3;  // + tile parity
+constexpr int kKqBarFull = 1;  // + buffer
+constexpr int kKqBarFree = 5;  // + buffer
 __device__ __forceinline__ void named_arrive(int id, int threads) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -187,7 +191,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
 // nibbles (sub-block 2t, scale a0 = d*sc, offset b0 = dmin*m), hi[k] the high
 // ones (sub-block 2t + 1: a1, b1); element 2k, 2k + 1 of a run are bytes
 // 2k, 2k + 1 of v.  Each weight is fma(a, q, -b): one rounding of the exact
-// d*sc*q - dmin*m, as in the row-per-warp kernel.
+// d*sc*q - dmin*m.
 __device__ __forceinline__ void q4_weights(const uint4 v, uint64_t a0, uint64_t nb0, uint64_t a1, uint64_t nb1,
                                            uint64_t (&lo)[8], uint64_t (&hi)[8]) {
     const uint32_t words[4] = {v.x, v.y, v.z, v.w};
@@ -280,13 +284,13 @@ __global__ void __launch_bounds__(kKqTileThreads, MINB)
     __syncthreads();
     // warp w's first block in tile t: blocks rotate by t * SB (mod 8)
     const int sb8 = SB & 7;
-    auto first_block = [&](int tile) { return (warp - (tile & 7) * sb8) & 7; };
-    auto blocks_of = [&](int tile) {
-        const int b0 = first_block(tile);
+    auto first_block = [&](int ti) { return (warp - (ti & 7) * sb8) & 7; };
+    auto blocks_of = [&](int ti) {
+        const int b0 = first_block(ti);
         return b0 < SB ? (SB - b0 + kKqWarps - 1) / kKqWarps : 0;
     };
     // producer iterator (lane 0): the (tile, block) of step `issued`
-    int p_ti = 0, p_bi = 0, p_nb = my_tiles > 0 ? blocks_of((int)blockIdx.x) : 0;
+    int p_ti = 0, p_bi = 0, p_nb = my_tiles > 0 ? blocks_of(0) : 0;
     int p_slot = 0, issued = 0;
     const uint64_t pw = policy_evict_first();
     bool broken = false;
@@ -295,11 +299,11 @@ __global__ void __launch_bounds__(kKqTileThreads, MINB)
         while (p_ti < my_tiles && p_bi >= p_nb) {
             ++p_ti;
             p_bi = 0;
-            p_nb = p_ti < my_tiles ? blocks_of((int)blockIdx.x + p_ti * (int)gridDim.x) : 0;
+            p_nb = p_ti < my_tiles ? blocks_of(p_ti) : 0;
         }
         if (p_ti >= my_tiles || broken) return;
         const int tile = (int)blockIdx.x + p_ti * (int)gridDim.x;
-        const int b = first_block(tile) + p_bi * kKqWarps;
+        const int b = first_block(p_ti) + p_bi * kKqWarps;
         if (lane == 0) {
             const uint32_t bar = bar0 + 8 * p_slot;
             const uint32_t dst = smem_u32(ring + p_slot * SBYTES);
@@ -322,7 +326,7 @@ __global__ void __launch_bounds__(kKqTileThreads, MINB)
     for (int ti = 0; ti < my_tiles; ++ti) {
         const int tile = (int)blockIdx.x + ti * (int)gridDim.x;
         const int row0 = tile * kKqRows;
-        const int nb = blocks_of(tile), bfirst = first_block(tile);
+        const int nb = blocks_of(ti), bfirst = first_block(ti);
         float acc[IT][NMAX];
 #pragma unroll
         for (int i = 0; i < IT; ++i)
@@ -441,10 +445,10 @@ __global__ void __launch_bounds__(kKqTileThreads, MINB)
             }
         }
         // ---- partial sums: the 8 lanes of a row, then the warps in order ----
-        const int p = ti & 1;
+        const int p = ti & (kKqRedBufs - 1);
         const int reducer = ti & 7;
-        if (ti >= 2 && warp != ((ti - 2) & 7)) named_barrier(kKqBarFree + p, kKqTileThreads);
-        float *rp = red + (size_t)p * kKqWarps * NMAX * kKqRows;
+        if (ti >= kKqRedBufs && warp != ((ti - kKqRedBufs) & 7)) named_barrier(kKqBarFree + p, kKqTileThreads);
+        float *rp = red + (size_t)p * kKqWarps * NMAX * kKqRows;  // [warp][n][row] of buffer p
 #pragma unroll
         for (int i = 0; i < IT; ++i)
 #pragma unroll
@@ -466,7 +470,7 @@ __global__ void __launch_bounds__(kKqTileThreads, MINB)
                 if (n < N && row < M && !broken) y[(size_t)n * M + row] = sum;
             }
             __syncwarp();
-            if (ti + 2 < my_tiles) named_arrive(kKqBarFree + p, kKqTileThreads);
+            if (ti + kKqRedBufs < my_tiles) named_arrive(kKqBarFree + p, kKqTileThreads);
         } else {
             named_arrive(kKqBarFull + p, kKqTileThreads);
         }
