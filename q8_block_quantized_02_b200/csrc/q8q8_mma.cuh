@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
             for (int ks = 0; ks < ksteps;
                  ++ks, ++it, slot = slot + 1 == a.stages ? 0 : slot + 1, phase ^= slot == 0 ? 1 : 0) {
                 uint8_t *st = smem + (size_t)slot * kMmaStageBytes;
-                const bool ok = mbar_wait_warp(full0 + 8 * slot, phase, abort_flag);
+                bool ok = mbar_wait_warp(full0 + 8 * slot, phase, abort_flag);
                 const float dx_cur = dx_next;
                 dx_next = dx_load(it + 1, ks + 1 == ksteps ? 0 : ks + 1);  // one stage ahead: it has a stage to land
                 if (ok && tab_thread) {
@@ -480,11 +480,15 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                 }
                 named_barrier(1, kMmaEpiThreads);
                 const int nb = min(kMmaSB, nblk - ks * kMmaSB);
-                for (int h = 0; h < kMmaHalves && ok; ++h) {
-                    const int j0 = h * kMmaHalfBlocks;
-                    uint32_t v[kMmaHalfBlocks * kMmaNPG];
+                // The TMEM loads of half h + 1 are issued before half h is
+                // computed, so their latency hides behind the arithmetic
+                // (tcgen05.wait::ld waits for every earlier load of the thread,
+                // so one batch is in flight at a time).
+                uint32_t va[kMmaHalfBlocks * kMmaNPG], vb[kMmaHalfBlocks * kMmaNPG];
+                // wait for half h's slot and issue its loads (no wait)
+                auto fetch = [&](int h, uint32_t(&v)[kMmaHalfBlocks * kMmaNPG]) -> bool {
                     const bool okh = mbar_wait_warp(tfull0 + 8 * ts, tph, abort_flag);
-                    if (okh && j0 < nb) {
+                    if (okh && h * kMmaHalfBlocks < nb) {
                         tc_fence_after();
 #pragma unroll
                         for (int jj = 0; jj < kMmaHalfBlocks; ++jj) {
@@ -494,6 +498,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                             else
                                 tmem_ld4_async(ta, v + jj * kMmaNPG);
                         }
+                    }
+                    return okh;
+                };
+                // wait for the loads in flight, then hand the slot back to the MMAs
+                auto land = [&](int h, uint32_t(&v)[kMmaHalfBlocks * kMmaNPG]) {
+                    if (h * kMmaHalfBlocks < nb) {
 #pragma unroll
                         for (int i = 0; i < kMmaHalfBlocks * kMmaNPG; i += 8) tmem_wait_ld8(v + i);
                         tc_fence_before();
@@ -501,13 +511,33 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(tempty0 + 8 * ts);
                     if (++ts == kMmaTSlots) { ts = 0; tph ^= 1; }
-                    if (!okh) break;
+                };
+                auto compute = [&](int h, const uint32_t(&v)[kMmaHalfBlocks * kMmaNPG]) {
                     // a full stage takes the branch-free path, so the four
                     // blocks' loads and arithmetic can interleave
                     if (nb == kMmaSB)
-                        compute_half(std::true_type{}, v, j0, nb, st);
+                        compute_half(std::true_type{}, v, h * kMmaHalfBlocks, nb, st);
                     else
-                        compute_half(std::false_type{}, v, j0, nb, st);
+                        compute_half(std::false_type{}, v, h * kMmaHalfBlocks, nb, st);
+                };
+                static_assert(kMmaHalves % 2 == 0, "halves go in pairs through va, vb");
+                if (ok) {
+                    ok = fetch(0, va);
+                    if (ok) land(0, va);
+                }
+#pragma unroll
+                for (int h = 0; h < kMmaHalves && ok; h += 2) {
+                    // va holds half h; vb takes half h + 1
+                    ok = fetch(h + 1, vb);
+                    if (!ok) break;
+                    compute(h, va);
+                    land(h + 1, vb);
+                    if (h + 2 < kMmaHalves) {
+                        ok = fetch(h + 2, va);
+                        if (!ok) break;
+                    }
+                    compute(h + 1, vb);
+                    if (h + 2 < kMmaHalves) land(h + 2, va);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty0 + 8 * slot);
