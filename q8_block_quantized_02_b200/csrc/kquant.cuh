@@ -144,12 +144,13 @@ __global__ void __launch_bounds__(kKqThreads) q6k_row_kernel(const uint8_t *__re
 // partials in warp order by one reducer warp per tile (warp i % 8 for the
 // CTA's i-th tile), so results are bit-identical from run to run (the
 // rotation depends on the grid, so they may differ between GPUs with
-// different SM counts).  The partials go through kKqRedBufs shared buffers
-// (tile i uses buffer i % 4) under named barriers: a warp arrives on the
-// buffer's "full" barrier and moves on; only the reducer waits there.  Before
-// writing tile i's partials a warp waits on the buffer's "free" barrier, on
-// which the reducer of tile i - 4 arrives once it has read them.  So no
-// computing warp waits for a slower one, except across four tiles.
+// different SM counts).  The partials go through RB shared buffers (4 at
+// N = 1, 2 at N = 2; tile i uses buffer i % RB) under named barriers: a warp
+// arrives on the buffer's "full" barrier and moves on; only the reducer waits
+// there.  Before writing tile i's partials a warp waits on the buffer's
+// "free" barrier, on which the reducer of tile i - RB arrives once it has
+// read them.  So no computing warp waits for a slower one, except across RB
+// tiles.
 constexpr int kKqWarps = 8;
 constexpr int kKqTileThreads = kKqWarps * 32;
 constexpr int kKqRows = 32;                      // rows per tile (8 per lane)
@@ -157,7 +158,10 @@ constexpr int kQ4StageBytes = kKqRows * 144;     // 4608
 constexpr int kQ6RowBytes = 208;                 // ql | qh | scales of one row
 constexpr int kQ6UnitBytes = kKqRows * kQ6RowBytes + kKqRows * 2;  // 6720
 constexpr int kQ6DOff = kKqRows * kQ6RowBytes;   // 6656
-constexpr int kKqRedBufs = 4;                    // partial-sum buffers (tiles in flight)
+// partial-sum buffers (tiles in flight): 4 at N = 1, 2 at N = 2 (so that two
+// CTAs fit on an SM)
+template <int NMAX>
+__host__ __device__ constexpr int kq_red_bufs() { return NMAX == 1 ? 4 : 2; }
 
 template <int FMT>
 __host__ __device__ constexpr int kq_stage_bytes() { return FMT == 4 ? kQ4StageBytes : kQ6UnitBytes; }
@@ -165,7 +169,9 @@ __host__ __device__ constexpr int kq_stage_bytes() { return FMT == 4 ? kQ4StageB
 template <int FMT, int NMAX, int STAGES>
 __host__ __device__ constexpr int kq_red_off() { return kKqWarps * STAGES * kq_stage_bytes<FMT>(); }
 template <int FMT, int NMAX, int STAGES>
-__host__ __device__ constexpr int kq_bar_off() { return kq_red_off<FMT, NMAX, STAGES>() + kKqRedBufs * kKqWarps * NMAX * kKqRows * 4; }
+__host__ __device__ constexpr int kq_bar_off() {
+    return kq_red_off<FMT, NMAX, STAGES>() + kq_red_bufs<NMAX>() * kKqWarps * NMAX * kKqRows * 4;
+}
 template <int FMT, int NMAX, int STAGES>
 __host__ __device__ constexpr int kq_smem_bytes() { return kq_bar_off<FMT, NMAX, STAGES>() + kKqWarps * STAGES * 8 + 16; }
 
@@ -445,9 +451,10 @@ __global__ void __launch_bounds__(kKqTileThreads, MINB)
             }
         }
         // ---- partial sums: the 8 lanes of a row, then the warps in order ----
-        const int p = ti & (kKqRedBufs - 1);
+        constexpr int RB = kq_red_bufs<NMAX>();
+        const int p = ti & (RB - 1);
         const int reducer = ti & 7;
-        if (ti >= kKqRedBufs && warp != ((ti - kKqRedBufs) & 7)) named_barrier(kKqBarFree + p, kKqTileThreads);
+        if (ti >= RB && warp != ((ti - RB) & 7)) named_barrier(kKqBarFree + p, kKqTileThreads);
         float *rp = red + (size_t)p * kKqWarps * NMAX * kKqRows;  // [warp][n][row] of buffer p
 #pragma unroll
         for (int i = 0; i < IT; ++i)
@@ -470,7 +477,7 @@ __global__ void __launch_bounds__(kKqTileThreads, MINB)
                 if (n < N && row < M && !broken) y[(size_t)n * M + row] = sum;
             }
             __syncwarp();
-            if (ti + kKqRedBufs < my_tiles) named_arrive(kKqBarFree + p, kKqTileThreads);
+            if (ti + RB < my_tiles) named_arrive(kKqBarFree + p, kKqTileThreads);
         } else {
             named_arrive(kKqBarFull + p, kKqTileThreads);
         }

@@ -613,9 +613,12 @@ static cudaError_t setup_moe_kernels(int max_smem) {
 static RegisterSetup g_reg_moe(setup_moe_kernels);
 
 // K-quant tile kernel variants: (format, N, stages, CTAs per SM).  Two CTAs
-// per SM at N = 1 (twice the warps to hide the dequantise-and-dot latency);
-// at N = 2 the registers allow one, with deeper rings.
-#define Q8_KQ_VARIANTS(X) X(4, 1, 3, 2) X(4, 2, 4, 1) X(6, 1, 2, 2) X(6, 2, 3, 1)
+// per SM (twice the warps to hide the dequantise-and-dot latency) wherever
+// there are tiles for them; at N = 2 that leaves room for two-stage rings
+// only, so matrices with fewer than two tiles per SM take one CTA per SM with
+// deeper rings (measured: 152064x3584 N = 2 Q4_K 161 against 180 us, Q6_K 151
+// against 179; 3584x18944 the other way round, 25.7 against 29.5).
+#define Q8_KQ_VARIANTS(X) X(4, 1, 3, 2) X(4, 2, 4, 1) X(4, 2, 2, 2) X(6, 1, 2, 2) X(6, 2, 3, 1) X(6, 2, 2, 2)
 static cudaError_t setup_q4k_kernels(int max_smem) {
     (void)max_smem;
 #define Q8_KQ_SETUP(F, NM, ST, MB)                                                                             \
@@ -861,11 +864,15 @@ static q8_status run_kquant(const void *W, const float *x, float *y, int64_t M, 
         const q8_status ms =
             make_map_3d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, 144, SB, M, 144, 144 * SB, 144, 1, kKqRows, true);
         if (ms != Q8_OK) return ms;
+        const bool many = ceil_div(M, kKqRows) >= 2 * (int64_t)dev->sms;
         for (int64_t n0 = 0; n0 < N; n0 += 2) {
             const int nn = (int)std::min<int64_t>(2, N - n0);
+            const float *xn = x + n0 * K;
+            float *yn = y + n0 * M;
             const q8_status st =
-                nn == 1 ? launch_kq_tile<4, 1, 3, 2>(map, w8, x + n0 * K, y + n0 * M, M, K, 1, dev->sms, stream, name)
-                        : launch_kq_tile<4, 2, 4, 1>(map, w8, x + n0 * K, y + n0 * M, M, K, 2, dev->sms, stream, name);
+                nn == 1 ? launch_kq_tile<4, 1, 3, 2>(map, w8, xn, yn, M, K, 1, dev->sms, stream, name)
+                : many  ? launch_kq_tile<4, 2, 2, 2>(map, w8, xn, yn, M, K, 2, dev->sms, stream, name)
+                        : launch_kq_tile<4, 2, 4, 1>(map, w8, xn, yn, M, K, 2, dev->sms, stream, name);
             if (st != Q8_OK) return st;
         }
         return Q8_OK;
@@ -890,11 +897,13 @@ static q8_status run_q6k_packed(const void *P, const float *x, float *y, int64_t
     const uint8_t *w8 = static_cast<const uint8_t *>(P);
     CUtensorMap unused;
     std::memset(&unused, 0, sizeof(unused));
+    const bool many = ceil_div(M, kKqRows) >= 2 * (int64_t)dev->sms;
     for (int64_t n0 = 0; n0 < N; n0 += 2) {
         const int nm = (int)std::min<int64_t>(2, N - n0);
         const float *xn = x + n0 * K;
         float *yn = y + n0 * M;
         const q8_status st = nm == 1 ? launch_kq_tile<6, 1, 2, 2>(unused, w8, xn, yn, M, K, 1, dev->sms, stream, name)
+                             : many  ? launch_kq_tile<6, 2, 2, 2>(unused, w8, xn, yn, M, K, 2, dev->sms, stream, name)
                                      : launch_kq_tile<6, 2, 3, 1>(unused, w8, xn, yn, M, K, 2, dev->sms, stream, name);
         if (st != Q8_OK) return st;
     }
