@@ -107,9 +107,10 @@ __global__ void __launch_bounds__(kKqThreads) q6k_row_kernel(const uint8_t *__re
 // a tile, warp w takes super-blocks b = w', w' + 8, ... (w' = w rotated by
 // i * SB for the CTA's i-th tile, so that over a few consecutive tiles every
 // warp gets the same share when SB is not a multiple of 8; rotating by the
-// global tile index would not, since a CTA's tiles are a grid apart).  A warp's (tile, block) steps stream through its
-// own ring of shared-memory stages, each holding one block of the tile's 32
-// rows and filled by one copy that lane 0 issues on the stage's mbarrier:
+// global tile index would not, since a CTA's tiles are a grid apart).  A
+// warp's (tile, block) steps stream through its own ring of shared-memory
+// stages, each holding one block of the tile's 32 rows and filled by one copy
+// that lane 0 issues on the stage's mbarrier:
 //   * Q4_K: the raw rows are 144 * SB bytes, so a 3-D TMA box {144 B, 1 block,
 //     32 rows} lands the stage as [32 rows][144 B] (rows past M read as zero);
 //   * Q6_K: raw 210-byte blocks start on 2-byte boundaries, out of reach of
@@ -125,10 +126,11 @@ __global__ void __launch_bounds__(kKqThreads) q6k_row_kernel(const uint8_t *__re
 //   * Q4_K piece u = 2t + h: weights 64t + 16h + i (low nibbles, sub-block 2t)
 //     and 64t + 32 + 16h + i (high nibbles, sub-block 2t + 1), i < 16.  Each
 //     weight is fma(d*sc, q, -dmin*m) (d*sc and dmin*m exact in fp32), one
-//     rounding relative to itself: factoring the
-//     sub-block's terms out of the sum would be cheaper, but its rounding
-//     would scale with d*sc*sum q x and dmin*m*sum x, not with sum |w x|, and
-//     the two cancel when the weights are near zero.
+//     rounding relative to itself: factoring the sub-block's terms out of
+//     the sum would be cheaper, but its rounding would scale with
+//     d*sc*sum q x and dmin*m*sum x, not with sum |w x|, and the two cancel
+//     when the weights are near zero.  Each lane decodes one sub-block's
+//     6-bit scale and min; the lanes of a row exchange them by shuffles.
 //   * Q6_K piece u = 4hh + 2a + j: ql bytes 64hh + 32a + 16j + i (i < 16) give
 //     weights 128hh + 32a + 16j + i (low nibble, 2 high bits from qh byte
 //     32hh + 16j + i at bit 2a, scale 8hh + 2a + j) and 128hh + 64 + 32a + 16j
@@ -137,7 +139,7 @@ __global__ void __launch_bounds__(kKqThreads) q6k_row_kernel(const uint8_t *__re
 //     scaled once by d * scale (exact): the rounding is relative to
 //     sum |w x| all the same, since w = d * scale * (q - 32) has no offset
 //     term that could cancel.
-// A 6-bit value becomes a float without a conversion: placed in the low
+// A 4- or 6-bit value becomes a float without a conversion: placed in the low
 // mantissa bits of 2^23 by a byte permute it gives 2^23 + q exactly, and one
 // paired subtract removes the bias.  Dots use packed f32x2 FMAs.
 // Row sums: the 8 lanes of a row by a shuffle tree, then the 8 warps'
@@ -165,7 +167,7 @@ __host__ __device__ constexpr int kq_red_bufs() { return NMAX == 1 ? 4 : 2; }
 
 template <int FMT>
 __host__ __device__ constexpr int kq_stage_bytes() { return FMT == 4 ? kQ4StageBytes : kQ6UnitBytes; }
-// Shared memory: rings [warp][stage] | partials [2][warp][NMAX][32] | barriers [warp][stage] | abort flag
+// Shared memory: rings [warp][stage] | partials [RB][warp][NMAX][32] | barriers [warp][stage] | abort flag
 template <int FMT, int NMAX, int STAGES>
 __host__ __device__ constexpr int kq_red_off() { return kKqWarps * STAGES * kq_stage_bytes<FMT>(); }
 template <int FMT, int NMAX, int STAGES>
