@@ -1,7 +1,8 @@
 """GPU parity of the K-quant GEMV (q8_q4k_gemv, q8_q6k_gemv: GGUF Q4_K / Q6_K
-super-blocks read in their raw layout) against the fp64 CPU oracle, through
-the C ABI.  Every packed field is random bytes, so all scale/min bit patterns
-and all nibble values occur.
+super-blocks read in their raw layout; q8_q6k_gemv_packed from the re-laid
+Q6_K units, with the pack layout and round trip) against the fp64 CPU oracle,
+through the C ABI.  Every packed field is random bytes, so all scale/min bit
+patterns and all nibble values occur.
 
 Tolerance: |y - y_ref| <= 1e-5 * sum_k |w_k x_k| per element, the GEMV bar."""
 from __future__ import annotations
@@ -36,8 +37,9 @@ def run(fmt, blocks, x, M, K):
 @pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
 @pytest.mark.parametrize("M,K,N", [(1, 256, 1), (13, 512, 2), (1000, 3584, 4), (37, 2048, 3),
                                    (3584, 18944, 1), (4096, 3584, 2),
-                                   # Q4_K at N <= 2 runs the row-tile kernel: tiles of 32
-                                   # rows (ragged last tile), blocks split over 8 warps
+                                   # Q4_K runs the tile kernel: tiles of 32 rows (ragged
+                                   # last tile), blocks split over 8 warps; SB = 1 leaves
+                                   # seven warps without a block
                                    (33, 256, 1), (4739, 2304, 1), (70, 4864, 2), (5000, 1024, 2)])
 def test_kquant_gemv_matches_oracle(fmt, M, K, N):
     blocks = q8gen.kquant_matrix(fmt, 5 * M + K + N, M, K)
