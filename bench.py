@@ -199,8 +199,9 @@ def gpu_configs(q8, torch, dev, stream):
     """Device time per call of the single GEMV (1152x896, seed 0), the 7B-class
     small-batch products (N = 1, 2, 4, 8, 16 through the default entry points,
     N = 3, 4, 8, 16 through the split ones), the Qwen1.5-MoE block (T = 1, 8)
-    and the Q8 x Q8 sweep (M = 4096, K in {896, 3584, 4864, 18944}, N in {1,
-    16}).  Calls walk distinct packed copies of each matrix covering several
+    the Q8 x Q8 sweep (M = 4096, K in {896, 3584, 4864, 18944}, N in {1,
+    16}) and the K-quant GEMV on the 7B lm_head shape (Q4_K raw, Q6_K packed;
+    N = 1, 2; block bytes 144 or 210 per 256 weights).  Calls walk distinct packed copies of each matrix covering several
     times the L2 (the same bytes, so only the cache behaviour differs), or
     distinct routings for the MoE block, so every call streams its weights
     from HBM.  Weight bytes are 34 per 32 weights."""
@@ -311,6 +312,27 @@ def gpu_configs(q8, torch, dev, stream):
                                     "weight_GBps": round(algorithmic_bytes(M, K) / us / 1e3, 1)}
         del ps
     out["q8q8_m4096"] = q8q8
+
+    # K-quant GEMV (f3) on the 7B lm_head shape: Q4_K on its raw blocks, Q6_K
+    # from its packed units; one copy of each (306 / 447 MB) exceeds the L2
+    M, K = 152064, 3584
+    for fmt, name in (("q4_k", "q4k"), ("q6_k", "q6k_packed")):
+        blocks = torch.from_numpy(q8gen.kquant_matrix(fmt, 777, M, K)).to(dev)
+        if fmt == "q6_k":
+            w8 = torch.empty(q8.q8_q6k_packed_bytes(M, K), dtype=torch.uint8, device=dev)
+            q8.q8_q6k_pack_weights(blocks, M, K, w8, stream=stream)
+            fn = q8.q8_q6k_gemv_packed
+        else:
+            w8 = blocks
+            fn = q8.q8_q4k_gemv
+        kq = {}
+        for N in (1, 2):
+            xd = torch.from_numpy(q8gen.activations(778 + N, N, K)).to(dev)
+            y = torch.empty((N, M), dtype=torch.float32, device=dev)
+            us = _graph_time_us(torch, stream, [lambda: fn(w8, xd, y, M, K, N, stream=stream)] * 4)
+            kq[f"N={N}"] = {"us_per_call": round(us, 2), "block_GBps": round(blocks.numel() / us / 1e3, 1)}
+        out[f"7b_lm_head_{M}x{K}_{name}"] = kq
+        del blocks, w8
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return out
@@ -364,6 +386,15 @@ def oracle_configs(threads):
             q[f"K={K},N={N}"] = round(timed(lambda: oracle.q8q8(g, xq, xd, S, K, want_dots=False, threads=threads))
                                       * 4096 / S, 1)
     out["q8q8_m4096"] = {"oracle_us_per_call": q, "oracle_sample": f"{S} output rows, scaled to 4096"}
+    for fmt, name in (("q4_k", "q4k"), ("q6_k", "q6k_packed")):
+        blocks = q8gen.kquant_matrix(fmt, 777, S, 3584)
+        res = {}
+        for N in (1, 2):
+            xs = q8gen.activations(778 + N, N, 3584)
+            res[f"N={N}"] = round(timed(lambda: oracle.kquant_gemv(fmt, blocks, xs, S, 3584, threads=threads))
+                                  * 152064 / S, 1)
+        out[f"7b_lm_head_152064x3584_{name}"] = {"oracle_us_per_call": res,
+                                                 "oracle_sample": f"{S} output rows (raw blocks), scaled to 152064"}
     return out
 
 
