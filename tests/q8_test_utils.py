@@ -89,3 +89,19 @@ def rows_subset(gguf: np.ndarray, M: int, K: int, rows: np.ndarray) -> np.ndarra
 
 def matrix(seed: int, M: int, K: int, N: int | None = None):
     return q8gen.q8_matrix(seed, M, K, N)
+
+
+def pack_q6k_reference(blocks, M, K):
+    """The packed layout as include/q8.h states it, written with numpy: unit
+    (t, b) of 6720 bytes; row i of tile t at byte 208 i holds raw bytes 0..207
+    of block b of matrix row 32t + i, bytes 6656 + 2i, + 1 its d; rows past M
+    zero."""
+    SB = K // 256
+    T = -(-M // 32)
+    raw = np.zeros((T * 32, SB, 210), np.uint8)
+    raw[:M] = blocks.reshape(M, SB, 210)
+    raw = raw.reshape(T, 32, SB, 210).transpose(0, 2, 1, 3)  # [t][b][i][210]
+    out = np.zeros((T, SB, 6720), np.uint8)
+    out[:, :, :6656] = raw[:, :, :, :208].reshape(T, SB, 6656)
+    out[:, :, 6656:] = raw[:, :, :, 208:].reshape(T, SB, 64)
+    return out.reshape(-1)
